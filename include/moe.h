@@ -1,0 +1,194 @@
+/*
+ * moe.h -- C ABI of the Kimi K2 routed mixture-of-experts layer, forward pass,
+ * on one NVIDIA B200 (sm_100a).
+ *
+ * The layer (definitions from the pages this library follows):
+ *   - Router: logits = x . W_g^T over n_routed_experts = 384 experts of
+ *     hidden_size = 7168 inputs, scoring_func = sigmoid,
+ *     topk_method = noaux_tc (an additive e_score_correction_bias is used to
+ *     choose experts only), n_group = topk_group = 1 (no group filter),
+ *     num_experts_per_tok = 8, norm_topk_prob = true (the 8 chosen unbiased
+ *     scores are normalised to sum 1), routed_scaling_factor = 2.827.
+ *     Source: "Kimi K2 Base" and "Kimi K2 0905" model cards, raw config.json
+ *     field tables.
+ *   - Experts: each routed expert and the shared expert
+ *     (n_shared_experts = 1) is the SwiGLU MLP
+ *     down_proj(silu(gate_proj(x)) * up_proj(x)), moe_intermediate_size 2048,
+ *     no biases, weights stored [out, in]. Source: "Kimi K2 · Down projection"
+ *     (OpenModelAtlas): the module formula, the parameter accounting table,
+ *     the "no bias" and "[out, in]" notes.
+ *   - Output: y[t] = sum_j w[t,j] * E_{id[t,j]}(x_t) + S(x_t), S the shared
+ *     expert with weight 1.
+ *   - FP8 variant: e4m3 weights, one fp32 scale per 128x128 block
+ *     (W = decode(q) * s), activation_scheme dynamic (per token, per 128
+ *     columns: s = amax/448, q = e4m3(v/s), nearest-even, saturating).
+ *     Source: the same page's config.json quantization_config excerpt.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named *_host are host memory; every other tensor pointer is a
+ *     device pointer on the handle's device (host pointers are also accepted
+ *     by moe_load_weights, which copies with cudaMemcpyDefault).
+ *   - All matrices are row-major and dense (no strides).
+ *   - BF16 is IEEE bfloat16 (uint16 storage); e4m3 is OCP FP8 E4M3 ("fn":
+ *     no infinities, max 448), one byte per value.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Work is enqueued on it and the calls return without waiting,
+ *     unless stated otherwise.
+ *   - The caller owns every buffer it passes; the library owns the copies it
+ *     makes and the handle's workspace, and frees them in moe_destroy.
+ *   - A handle is used by one host thread at a time. Forwards on one handle
+ *     share its workspace, so they must be ordered on one stream.
+ *   - Errors: a call returns a negative moe_status_t and launches nothing
+ *     when it detects a bad argument on the host. Problems found by a kernel
+ *     (a wait that ran out of time, a forced expert id out of range) set a
+ *     device status word; it is read by moe_get_device_status, or by a
+ *     forward called with MOE_FLAG_SYNC_CHECK. No kernel traps or asserts.
+ */
+#ifndef SPARSE_MOE_SIGMOID_B200_MOE_H
+#define SPARSE_MOE_SIGMOID_B200_MOE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1, /* a null pointer, a size out of range, aliasing */
+  MOE_ERR_UNSUPPORTED = -2, /* a config outside what the kernels implement */
+  MOE_ERR_OOM = -3,         /* device allocation failed */
+  MOE_ERR_CUDA = -4,        /* a CUDA runtime call failed (see moe_last_error) */
+  MOE_ERR_DEVICE = -5,      /* a kernel reported a problem in the status word */
+  MOE_ERR_TIMEOUT = -6,     /* a kernel wait ran out of time and returned */
+  MOE_ERR_STATE = -7        /* e.g. forward before moe_load_weights */
+} moe_status_t;
+
+typedef enum {
+  MOE_WEIGHT_BF16 = 0,           /* expert weights BF16 */
+  MOE_WEIGHT_FP8_E4M3_BLOCK = 1  /* e4m3 + fp32 scale per 128x128 block */
+} moe_weight_format_t;
+
+typedef enum { MOE_SCORING_SIGMOID = 0 } moe_scoring_func_t;
+typedef enum { MOE_TOPK_NOAUX_TC = 0 } moe_topk_method_t;
+typedef enum { MOE_ACTIVATION_DYNAMIC = 0 } moe_activation_scheme_t;
+
+/* Layer configuration. Field names follow the model's config.json. */
+typedef struct {
+  int32_t hidden_size;            /* d: 7168 for K2; multiple of 128, <= 16384 */
+  int32_t moe_intermediate_size;  /* f: 2048 for K2; multiple of 128, <= 8192 */
+  int32_t n_routed_experts;       /* E: 384 for K2; 1..512 */
+  int32_t num_experts_per_tok;    /* k: 8 for K2; 1..min(E, 32) */
+  int32_t n_shared_experts;       /* 1 for K2; 0..8 (intermediate f * n_shared) */
+  int32_t n_group;                /* must be 1 (K2) */
+  int32_t topk_group;             /* must be 1 (K2) */
+  int32_t norm_topk_prob;         /* 1 (K2): normalise the k scores; 0: do not */
+  float routed_scaling_factor;    /* 2.827 for K2 */
+  int32_t scoring_func;           /* MOE_SCORING_SIGMOID */
+  int32_t topk_method;            /* MOE_TOPK_NOAUX_TC */
+  int32_t weight_format;          /* moe_weight_format_t */
+  int32_t weight_block_size[2];   /* {128, 128}; checked for the FP8 format */
+  int32_t activation_scheme;      /* MOE_ACTIVATION_DYNAMIC */
+  int64_t max_tokens;             /* largest T a forward will get; sizes the workspace */
+} moe_config_t;
+
+/* Weights handed to moe_load_weights (caller-owned; copied by the call).
+ * E = n_routed_experts, d = hidden_size, f = moe_intermediate_size,
+ * fs = f * n_shared_experts. Element type of *_proj: BF16 or e4m3 by the
+ * config's weight_format. Layout [out, in]. */
+typedef struct {
+  const float* router_weight;           /* [E, d] fp32 */
+  const float* e_score_correction_bias; /* [E] fp32 */
+  const void* gate_proj;                /* [E, f, d] */
+  const void* up_proj;                  /* [E, f, d] */
+  const void* down_proj;                /* [E, d, f] */
+  const float* gate_scale;              /* FP8: [E, f/128, d/128] fp32, else NULL */
+  const float* up_scale;                /* FP8: [E, f/128, d/128] */
+  const float* down_scale;              /* FP8: [E, d/128, f/128] */
+  const void* shared_gate_proj;         /* [fs, d]  (NULL when n_shared_experts = 0) */
+  const void* shared_up_proj;           /* [fs, d] */
+  const void* shared_down_proj;         /* [d, fs] */
+  const float* shared_gate_scale;       /* FP8: [fs/128, d/128] */
+  const float* shared_up_scale;         /* FP8: [fs/128, d/128] */
+  const float* shared_down_scale;       /* FP8: [d/128, fs/128] */
+} moe_weights_t;
+
+/* moe_forward_opts_t.flags */
+#define MOE_FLAG_SYNC_CHECK 0x1u /* synchronise the stream and read the device status word */
+
+typedef struct {
+  int32_t* topk_ids_out;          /* optional device [T, k]: chosen experts, key-descending */
+  float* topk_weights_out;        /* optional device [T, k]: their weights (sum 2.827) */
+  const int32_t* forced_topk_ids; /* optional device [T, k]: use these experts instead of
+                                     selecting (weights still from the unbiased scores);
+                                     ids must be distinct per token and < E, else the
+                                     status word gets MOE_DEVICE_BAD_EXPERT_ID */
+  uint32_t flags;                 /* MOE_FLAG_* */
+} moe_forward_opts_t;
+
+/* Device status word bits (moe_get_device_status) */
+#define MOE_DEVICE_WAIT_TIMEOUT 0x1u   /* a pipeline wait in a GEMM kernel ran out of time */
+#define MOE_DEVICE_BAD_EXPERT_ID 0x2u  /* a forced expert id was out of range or repeated */
+
+typedef struct moe_handle moe_handle_t;
+
+/* Fill *cfg with the Kimi K2 layer (values above) and max_tokens = 8192. */
+moe_status_t moe_config_init_k2(moe_config_t* cfg);
+
+/* Validate cfg, select `device`, allocate the handle's weight buffers and a
+ * workspace for up to cfg->max_tokens tokens. Unsupported values
+ * (n_group != 1, other scoring or top-k methods, sizes not multiples of 128)
+ * return MOE_ERR_UNSUPPORTED. Synchronous. */
+moe_status_t moe_create(const moe_config_t* cfg, int device, moe_handle_t** out);
+
+/* Copy the weights into the handle's buffers (the shared expert becomes
+ * n_shared_experts extra experts of intermediate size f each, which sum to
+ * the same output). Ordered on `stream`; the caller's buffers may be freed
+ * once the stream has reached this point. */
+moe_status_t moe_load_weights(moe_handle_t* h, const moe_weights_t* w, void* stream);
+
+/* y = MoE(x) for T tokens. x: device BF16 [T, d]; y: device BF16 [T, d]
+ * (must not overlap x). T = 0 is a no-op. T > max_tokens is
+ * MOE_ERR_INVALID_ARG. Asynchronous on `stream` unless opts->flags has
+ * MOE_FLAG_SYNC_CHECK. opts may be NULL. */
+moe_status_t moe_forward(moe_handle_t* h, const void* x, int64_t T, void* y,
+                         const moe_forward_opts_t* opts, void* stream);
+
+/* The same forward from and to host memory: copies x_host (BF16 [T, d]) to
+ * the device, runs moe_forward, copies y back into y_host, all on `stream`,
+ * then synchronises the stream. Page-locked host buffers give the fastest
+ * copies; pageable ones work. */
+moe_status_t moe_forward_host(moe_handle_t* h, const void* x_host, int64_t T, void* y_host,
+                              const moe_forward_opts_t* opts, void* stream);
+
+/* Synchronise the handle's device, return the device status word in
+ * *flags (MOE_DEVICE_* bits) and clear it. */
+moe_status_t moe_get_device_status(moe_handle_t* h, uint32_t* flags);
+
+/* Per-phase timing. moe_profile_enable(h, n) makes the next n forwards
+ * record CUDA events between their phases (n = 0 turns it off).
+ * moe_profile_read waits for them and writes ms[i * MOE_NUM_PHASES + p] for
+ * forward i and phase p, at most `cap` floats; *n_forwards gets the count. */
+#define MOE_NUM_PHASES 7
+/* phase order: 0 router logits, 1 router top-k, 2 route scan, 3 dispatch,
+ * 4 gate/up GEMM + SwiGLU, 5 down GEMM, 6 combine */
+moe_status_t moe_profile_enable(moe_handle_t* h, int32_t max_forwards);
+moe_status_t moe_profile_read(moe_handle_t* h, float* ms, int32_t cap, int32_t* n_forwards);
+
+/* Number of kernels this handle has launched so far. */
+int64_t moe_launch_count(const moe_handle_t* h);
+
+/* Free everything the handle owns. NULL is a no-op. Synchronises the device. */
+void moe_destroy(moe_handle_t* h);
+
+/* Static text for a status code. */
+const char* moe_status_string(moe_status_t s);
+
+/* Detail of the last error on this handle (empty string if none). */
+const char* moe_last_error(const moe_handle_t* h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_MOE_SIGMOID_B200_MOE_H */

@@ -98,7 +98,7 @@ def encode(values: np.ndarray) -> np.ndarray:
     out = np.zeros(v.shape, dtype=np.int64)
 
     sub = a < 2.0 ** -6
-    n_sub = np.rint(a * 2.0 ** 9)  # numpy rint rounds half to even
+    n_sub = np.rint(np.minimum(a, 2.0 ** -6) * 2.0 ** 9)  # numpy rint rounds half to even
     out = np.where(sub, n_sub.astype(np.int64), out)  # n_sub == 8 -> 0x08 = smallest normal
 
     with np.errstate(divide="ignore", invalid="ignore"):

@@ -1,0 +1,291 @@
+// Token-to-expert dispatch and the weighted combine.
+//
+// The pages describe 384 independent experts that each see only their own
+// tokens ("Kimi K2 · Down projection": 384 routed experts, each its own
+// SwiGLU MLP); how tokens are grouped per expert is this library's design:
+//
+//   rows: every (token, slot) pair routed to expert e gets one row, and the
+//   rows of expert e are contiguous [offsets[e], offsets[e+1]) in ascending
+//   token order. The shared expert (split into n_shared groups of
+//   moe_intermediate_size each) follows as groups E.., each holding all T
+//   tokens in order.
+//
+// route_scan_kernel (one CTA): exclusive scan of the per-group row counts
+//   into offsets; the GEMM work-unit prefix for both grouped GEMMs; and for
+//   every expert the running popcount of its token bitmap words, so a pair's
+//   rank inside its expert is one popcount away.
+// dispatch_kernel: one warp per row. It places the pair (pair_row,
+//   row_token) and copies the token's x row into the gathered matrix with
+//   16-byte loads and stores. In the FP8 format it quantises on the way:
+//   per 128 columns s = amax/448 and q = e4m3(x/s), both divisions
+//   correctly rounded, conversion nearest-even and saturating.
+// combine_kernel: y[t] = sum_j w[t,j] * out[row(t,j)] + sum_s out[shared
+//   row(s,t)] in fp32, in slot order, rounded once to BF16.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "internal.h"
+
+namespace smoe {
+
+static int pick_bn(double want, const int* cands, int n) {
+  for (int i = 0; i < n; ++i)
+    if (cands[i] >= want) return cands[i];
+  return cands[n - 1];
+}
+
+GemmPlan plan_gate_up(const Dims& dm, int64_t T) {
+  static const int bf16_bn[] = {16, 32, 64, 128};
+  static const int fp8_bn[] = {16, 32, 64};
+  const double avg = static_cast<double>(T) * dm.k / dm.E;
+  GemmPlan p;
+  p.bn = dm.fp8 ? pick_bn(avg * 1.5, fp8_bn, 3) : pick_bn(avg * 1.5, bf16_bn, 4);
+  p.m_tiles = dm.f / kBlock;
+  p.k_blocks = dm.fp8 ? dm.d / 128 : dm.d / 64;
+  return p;
+}
+
+GemmPlan plan_down(const Dims& dm, int64_t T) {
+  static const int bf16_bn[] = {16, 32, 64, 128, 256};
+  static const int fp8_bn[] = {16, 32, 64, 128};
+  const double avg = static_cast<double>(T) * dm.k / dm.E;
+  GemmPlan p;
+  p.bn = dm.fp8 ? pick_bn(avg * 1.5, fp8_bn, 4) : pick_bn(avg * 1.5, bf16_bn, 5);
+  p.m_tiles = dm.d / kBlock;
+  p.k_blocks = dm.fp8 ? dm.f / 128 : dm.f / 64;
+  return p;
+}
+
+// --------------------------------------------------------------- route scan
+constexpr int kScanThreads = 1024;
+
+__device__ __forceinline__ int block_exclusive_scan(int v, int* tmp, int* total) {
+  // Hillis-Steele inclusive scan over the CTA, then shift to exclusive.
+  const int tid = threadIdx.x;
+  tmp[tid] = v;
+  __syncthreads();
+  for (int off = 1; off < kScanThreads; off <<= 1) {
+    const int add = tid >= off ? tmp[tid - off] : 0;
+    __syncthreads();
+    tmp[tid] += add;
+    __syncthreads();
+  }
+  const int incl = tmp[tid];
+  *total = tmp[kScanThreads - 1];
+  __syncthreads();
+  return incl - v;
+}
+
+__global__ void __launch_bounds__(kScanThreads) route_scan_kernel(
+    const int32_t* __restrict__ counts, int E, int ns, int T, const uint32_t* __restrict__ bitmap,
+    int W, int32_t* __restrict__ word_prefix, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ unit_base, int bn1, int mt1, int bn2, int mt2) {
+  __shared__ int tmp[kScanThreads];
+  const int G = E + ns;
+  const int g = threadIdx.x;  // G <= kMaxExperts + 8 < 1024
+  int c = 0;
+  if (g < E) c = counts[g];
+  else if (g < G) c = T;
+  const int u1 = mt1 * ((c + bn1 - 1) / bn1);
+  const int u2 = mt2 * ((c + bn2 - 1) / bn2);
+  int tot;
+  const int o = block_exclusive_scan(c, tmp, &tot);
+  if (g <= G) offsets[g] = o;
+  const int b1 = block_exclusive_scan(u1, tmp, &tot);
+  if (g <= G) unit_base[g] = b1;
+  const int b2 = block_exclusive_scan(u2, tmp, &tot);
+  if (g <= G) unit_base[(G + 1) + g] = b2;
+
+  // per-expert running popcount of the token bitmap
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = warp; e < E; e += kScanThreads / 32) {
+    int run = 0;
+    for (int w0 = 0; w0 < W; w0 += 32) {
+      const int w = w0 + lane;
+      const int v = w < W ? __popc(bitmap[(size_t)e * W + w]) : 0;
+      int incl = v;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += n;
+      }
+      if (w < W) word_prefix[(size_t)e * W + w] = run + incl - v;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  }
+}
+
+cudaError_t launch_route_scan(moe_handle* h, int T, const GemmPlan& p1, const GemmPlan& p2,
+                              cudaStream_t s) {
+  const Dims& dm = h->dims;
+  const int W = static_cast<int>((dm.Tmax + 31) / 32);
+  route_scan_kernel<<<1, kScanThreads, 0, s>>>(h->ws.counts, dm.E, dm.ns, T, h->ws.bitmap, W,
+                                               h->ws.word_prefix, h->ws.offsets, h->ws.unit_base,
+                                               p1.bn, p1.m_tiles, p2.bn, p2.m_tiles);
+  h->launches++;
+  return cudaGetLastError();
+}
+
+// ----------------------------------------------------------------- dispatch
+__device__ __forceinline__ int place_row(int i, int T, int k, int E, const int32_t* ids,
+                                         const uint32_t* bitmap, const int32_t* word_prefix,
+                                         const int32_t* offsets, int W, int* tok) {
+  const int nrouted = T * k;
+  if (i < nrouted) {
+    const int t = i / k;
+    const int e = ids[i];
+    const int w = t >> 5;
+    const uint32_t below = bitmap[(size_t)e * W + w] & ((1u << (t & 31)) - 1u);
+    *tok = t;
+    return offsets[e] + word_prefix[(size_t)e * W + w] + __popc(below);
+  }
+  const int s = (i - nrouted) / T;
+  const int t = (i - nrouted) % T;
+  *tok = t;
+  return offsets[E + s] + t;
+}
+
+__global__ void __launch_bounds__(256) dispatch_bf16_kernel(
+    const __nv_bfloat16* __restrict__ x, int T, int d, int k, int E, int items,
+    const int32_t* __restrict__ ids, const uint32_t* __restrict__ bitmap,
+    const int32_t* __restrict__ word_prefix, const int32_t* __restrict__ offsets, int W,
+    int32_t* __restrict__ pair_row, int32_t* __restrict__ row_token,
+    __nv_bfloat16* __restrict__ xp) {
+  const int lane = threadIdx.x & 31;
+  const int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (i >= items) return;
+  int t;
+  const int row = place_row(i, T, k, E, ids, bitmap, word_prefix, offsets, W, &t);
+  if (lane == 0) {
+    if (i < T * k) pair_row[i] = row;
+    row_token[row] = t;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+  uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)row * d);
+  const int n16 = d / 8;
+  for (int c = lane; c < n16; c += 32) dst[c] = __ldg(src + c);
+}
+
+__global__ void __launch_bounds__(256) dispatch_fp8_kernel(
+    const __nv_bfloat16* __restrict__ x, int T, int d, int k, int E, int items,
+    const int32_t* __restrict__ ids, const uint32_t* __restrict__ bitmap,
+    const int32_t* __restrict__ word_prefix, const int32_t* __restrict__ offsets, int W,
+    int32_t* __restrict__ pair_row, int32_t* __restrict__ row_token, uint8_t* __restrict__ xq,
+    float* __restrict__ xs) {
+  const int lane = threadIdx.x & 31;
+  const int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (i >= items) return;
+  int t;
+  const int row = place_row(i, T, k, E, ids, bitmap, word_prefix, offsets, W, &t);
+  if (lane == 0) {
+    if (i < T * k) pair_row[i] = row;
+    row_token[row] = t;
+  }
+  const int ngroups = d / 128;
+  // each half-warp quantises one 128-column group: 16 lanes x 8 values
+  for (int g0 = 0; g0 < ngroups; g0 += 2) {
+    const int gi = g0 + (lane >> 4);
+    const bool active = gi < ngroups;
+    const int col = gi * 128 + (lane & 15) * 8;
+    float v[8];
+    float amax = 0.f;
+    if (active) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d + col));
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f2 = __bfloat1622float2(p[j]);
+        v[2 * j] = f2.x;
+        v[2 * j + 1] = f2.y;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    }
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1)
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (active) {
+      const float sa = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+      uint32_t packed[2];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float2 q;
+        q.x = __fdiv_rn(v[2 * j], sa);
+        q.y = __fdiv_rn(v[2 * j + 1], sa);
+        const __nv_fp8x2_storage_t b = __nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
+        if (j & 1) packed[j >> 1] |= static_cast<uint32_t>(b) << 16;
+        else packed[j >> 1] = static_cast<uint32_t>(b);
+      }
+      *reinterpret_cast<uint2*>(xq + (size_t)row * d + col) = make_uint2(packed[0], packed[1]);
+      if ((lane & 15) == 0) xs[(size_t)row * ngroups + gi] = sa;
+    }
+  }
+}
+
+cudaError_t launch_dispatch(moe_handle* h, const void* x, int T, cudaStream_t s) {
+  const Dims& dm = h->dims;
+  const int W = static_cast<int>((dm.Tmax + 31) / 32);
+  const int items = T * (dm.k + dm.ns);
+  const int blocks = static_cast<int>(((int64_t)items * 32 + 255) / 256);
+  if (dm.fp8) {
+    dispatch_fp8_kernel<<<blocks, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), T, dm.d, dm.k, dm.E, items, h->ws.ids,
+        h->ws.bitmap, h->ws.word_prefix, h->ws.offsets, W, h->ws.pair_row, h->ws.row_token,
+        static_cast<uint8_t*>(h->ws.xp), h->ws.xs);
+  } else {
+    dispatch_bf16_kernel<<<blocks, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), T, dm.d, dm.k, dm.E, items, h->ws.ids,
+        h->ws.bitmap, h->ws.word_prefix, h->ws.offsets, W, h->ws.pair_row, h->ws.row_token,
+        static_cast<__nv_bfloat16*>(h->ws.xp));
+  }
+  h->launches++;
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ combine
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ out,
+                                                      const int32_t* __restrict__ pair_row,
+                                                      const float* __restrict__ wts,
+                                                      const int32_t* __restrict__ offsets, int T,
+                                                      int d, int k, int E, int ns,
+                                                      __nv_bfloat16* __restrict__ y) {
+  const int t = blockIdx.x;
+  const int c = (blockIdx.y * blockDim.x + threadIdx.x) * 4;
+  if (c >= d) return;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = 0; j < k; ++j) {
+    const int row = pair_row[(size_t)t * k + j];
+    const float w = wts[(size_t)t * k + j];
+    const float4 v = __ldg(reinterpret_cast<const float4*>(out + (size_t)row * d + c));
+    acc.x = fmaf(w, v.x, acc.x);
+    acc.y = fmaf(w, v.y, acc.y);
+    acc.z = fmaf(w, v.z, acc.z);
+    acc.w = fmaf(w, v.w, acc.w);
+  }
+  for (int s = 0; s < ns; ++s) {
+    const int row = offsets[E + s] + t;
+    const float4 v = __ldg(reinterpret_cast<const float4*>(out + (size_t)row * d + c));
+    acc.x += v.x;
+    acc.y += v.y;
+    acc.z += v.z;
+    acc.w += v.w;
+  }
+  __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+  __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+  uint2 pk;
+  pk.x = *reinterpret_cast<uint32_t*>(&lo);
+  pk.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(y + (size_t)t * d + c) = pk;
+}
+
+cudaError_t launch_combine(moe_handle* h, void* y, int T, cudaStream_t s) {
+  const Dims& dm = h->dims;
+  dim3 grid(T, (dm.d / 4 + 255) / 256);
+  combine_kernel<<<grid, 256, 0, s>>>(h->ws.out, h->ws.pair_row, h->ws.wts, h->ws.offsets, T,
+                                      dm.d, dm.k, dm.E, dm.ns,
+                                      static_cast<__nv_bfloat16*>(y));
+  h->launches++;
+  return cudaGetLastError();
+}
+
+}  // namespace smoe

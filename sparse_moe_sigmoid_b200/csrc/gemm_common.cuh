@@ -1,0 +1,68 @@
+// Pieces shared by the BF16 and FP8 grouped GEMM kernels: the work-unit
+// decoding and the shared-memory carve-up.
+//
+// Work decomposition (both GEMMs of the expert MLP): the output of group g
+// (an expert, or a slice of the shared expert) is a [features x rows]
+// matrix, rows = the tokens routed to g. It is cut into tiles of 128
+// features x BN rows. A unit is one such tile; units are numbered group by
+// group, feature tile by feature tile, row tile innermost, so units that use
+// the same 128-row weight slab are adjacent and run at the same time on
+// neighbouring CTAs, which then read the slab from HBM once and from L2
+// after that. CTA c takes units c, c + gridDim.x, ... (persistent grid).
+#pragma once
+
+#include <stdint.h>
+
+namespace smoe {
+
+struct Unit {
+  int g;       // group (expert)
+  int mt;      // 128-feature tile
+  int row0;    // first row of the row tile
+  int nvalid;  // rows of the tile that belong to g (1..BN)
+};
+
+struct GemmArgs {
+  const int32_t* offsets;    // [G+1]
+  const int32_t* unit_base;  // [G+1] prefix of units per group
+  int G;
+  int m_tiles;
+  int k_blocks;
+  int bn;
+  void* out;                 // gate/up: h [R][ld]; down: fp32 out [R][ld]
+  int ld;
+  float* out_scale;          // FP8 gate/up: h scales [R][f/128]
+  const float* w_scale0;     // FP8: weight block scales of A0 [G][m_tiles][k_blocks]
+  const float* w_scale1;     // FP8 gate/up: of A1
+  const float* act_scale;    // FP8: activation scales [R][k_blocks]
+  uint32_t* status;
+};
+
+__device__ __forceinline__ Unit decode_unit(int u, const GemmArgs& a, int BN) {
+  // last group whose first unit is <= u (empty groups own no units)
+  int lo = 0, hi = a.G;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(a.unit_base + mid) <= u) lo = mid;
+    else hi = mid;
+  }
+  Unit un;
+  un.g = lo;
+  const int r0 = __ldg(a.offsets + lo);
+  const int cnt = __ldg(a.offsets + lo + 1) - r0;
+  const int nt = (cnt + BN - 1) / BN;
+  const int local = u - __ldg(a.unit_base + lo);
+  un.mt = local / nt;
+  const int ti = local - un.mt * nt;
+  un.row0 = r0 + ti * BN;
+  un.nvalid = min(BN, cnt - ti * BN);
+  return un;
+}
+
+__host__ __device__ constexpr int pow2_at_least(int v, int lo) {
+  int p = lo;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+}  // namespace smoe

@@ -1,0 +1,112 @@
+// Internal declarations shared by the library's .cu files (not installed).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "../../include/moe.h"
+
+namespace smoe {
+
+constexpr int kBlock = 128;       // FP8 block edge and GEMM M tile
+constexpr int kMaxTopK = 32;
+constexpr int kMaxExperts = 512;
+constexpr int kRouterTile = 64;   // router tile: 64 tokens x 64 experts
+constexpr int kRouterKTile = 32;
+
+// Sizes derived from the config, fixed per handle.
+struct Dims {
+  int d, f, E, k, ns, G;  // G = E + ns groups (shared expert split into ns groups)
+  bool fp8;
+  int64_t Tmax, Rmax;     // Rmax = Tmax * (k + ns)
+};
+
+// One grouped GEMM launch's shape choice.
+struct GemmPlan {
+  int bn;       // token rows per tile (MMA N upper bound)
+  int m_tiles;  // output features / 128
+  int k_blocks; // reduction / kernel K step
+};
+
+struct Workspace {
+  float* logits_part = nullptr;   // [splits][T][E]
+  int32_t* ids = nullptr;         // [T][k]
+  float* wts = nullptr;           // [T][k]
+  int32_t* counts = nullptr;      // [E]            (zeroed per forward)
+  uint32_t* bitmap = nullptr;     // [E][W] token bitmaps, W = ceil(Tmax/32) (zeroed per forward)
+  int32_t* word_prefix = nullptr; // [E][W]
+  int32_t* offsets = nullptr;     // [G+1] row offset of each group
+  int32_t* unit_base = nullptr;   // [2][G+1] per-GEMM unit prefix
+  int32_t* pair_row = nullptr;    // [T*k] row of each (token, slot)
+  int32_t* row_token = nullptr;   // [Rmax] token of each row
+  void* xp = nullptr;             // [Rmax][d] gathered rows, BF16 or e4m3
+  float* xs = nullptr;            // [Rmax][d/128] FP8 activation scales
+  void* hbuf = nullptr;           // [Rmax][f] SwiGLU output, BF16 or e4m3
+  float* hs = nullptr;            // [Rmax][f/128] FP8 scales of h
+  float* out = nullptr;           // [Rmax][d] fp32 per-row expert outputs
+  uint32_t* status = nullptr;     // device status word
+  void* x_stage = nullptr;        // [Tmax][d] BF16 staging for the host entry point
+  void* y_stage = nullptr;        // [Tmax][d]
+  size_t zero_bytes = 0;          // bytes of the counts+bitmap region cleared per forward
+};
+
+struct Weights {
+  float* router = nullptr;  // [E][d]
+  float* bias = nullptr;    // [E]
+  void* gate = nullptr;     // [G][f][d]
+  void* up = nullptr;       // [G][f][d]
+  void* down = nullptr;     // [G][d][f]
+  float* gate_s = nullptr;  // [G][f/128][d/128]
+  float* up_s = nullptr;
+  float* down_s = nullptr;  // [G][d/128][f/128]
+  bool loaded = false;
+};
+
+}  // namespace smoe
+
+struct moe_handle {
+  moe_config_t cfg;
+  int device = 0;
+  int num_sms = 148;
+  smoe::Dims dims{};
+  smoe::Weights w;
+  smoe::Workspace ws;
+  // TMA descriptors: weights (one per projection) and the two activation
+  // matrices, the latter once per supported row-tile height (16 << i)
+  CUtensorMap tm_gate, tm_up, tm_down;
+  CUtensorMap tm_xp[5], tm_h[5];
+  int router_max_splits = 1;
+  int64_t launches = 0;
+  std::string last_error;
+  // per-phase profiling
+  std::vector<cudaEvent_t> prof_events;
+  int prof_cap = 0, prof_next = 0;
+};
+
+namespace smoe {
+
+// router.cu
+int router_splits(const Dims& dm, int64_t T, int num_sms);
+cudaError_t launch_router_logits(moe_handle* h, const void* x, int T, int splits, cudaStream_t s);
+cudaError_t launch_router_topk(moe_handle* h, int T, int splits, const int32_t* forced,
+                               cudaStream_t s, int32_t* ids_out, float* wts_out);
+// dispatch.cu
+GemmPlan plan_gate_up(const Dims& dm, int64_t T);
+GemmPlan plan_down(const Dims& dm, int64_t T);
+cudaError_t launch_route_scan(moe_handle* h, int T, const GemmPlan& p1, const GemmPlan& p2,
+                              cudaStream_t s);
+cudaError_t launch_dispatch(moe_handle* h, const void* x, int T, cudaStream_t s);
+cudaError_t launch_combine(moe_handle* h, void* y, int T, cudaStream_t s);
+// gemm_bf16.cu / gemm_fp8.cu
+cudaError_t launch_gemm_bf16(moe_handle* h, bool gated, const GemmPlan& p, cudaStream_t s);
+cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaStream_t s);
+int bn_index(int bn);
+// api.cu
+bool make_tmap(CUtensorMap* m, CUtensorMapDataType dt, int rank, void* base, const uint64_t* dims,
+               const uint64_t* strides_bytes, const uint32_t* box, std::string* err);
+
+}  // namespace smoe

@@ -1,0 +1,272 @@
+// Router of the K2 MoE layer: logits, sigmoid scores, noaux_tc biased top-k,
+// normalisation and routed scaling.
+//
+// Config fields (scoring_func sigmoid, topk_method noaux_tc, n_group 1,
+// num_experts_per_tok 8, norm_topk_prob true, routed_scaling_factor 2.827):
+// "Kimi K2 Base" / "Kimi K2 0905" model cards, raw config field tables.
+//
+// Kernel 1 (router_logits_kernel): logits = x . W_g^T in fp32 on CUDA cores.
+//   The router weight is fp32, and tensor-core TF32 would move logits by
+//   ~1e-3, enough to change which experts win; so this is an exact-product
+//   fp32 FMA GEMM tiled 64 tokens x 64 experts. Small T splits the hidden
+//   dimension into `splits` slices so the grid covers the SMs; the partial
+//   sums land in [splits][T][E] and are added in slice order by kernel 2,
+//   which keeps the result deterministic.
+// Kernel 2 (router_topk_kernel): one warp per token. Lane l holds experts
+//   l, l+32, ...; it adds the partials, takes the sigmoid, forms the key
+//   score + bias, and the warp extracts the k largest keys (ties to the lower
+//   expert index) by k rounds of a shuffle arg-max. The weights use the
+//   unbiased scores: w = score / sum(selected scores) * 2.827. It also counts
+//   tokens per expert and sets the token's bit in the expert's bitmap, which
+//   the dispatch uses to place each (token, slot) pair.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "internal.h"
+
+namespace smoe {
+
+int router_splits(const Dims& dm, int64_t T, int num_sms) {
+  const int64_t tiles = ((dm.E + kRouterTile - 1) / kRouterTile) *
+                        ((T + kRouterTile - 1) / kRouterTile);
+  int64_t want = (2 * num_sms + tiles - 1) / tiles;
+  int64_t max_splits = dm.d / kRouterKTile;
+  if (want < 1) want = 1;
+  if (want > max_splits) want = max_splits;
+  // each slice is a multiple of the 32-wide K tile
+  int64_t kps = (dm.d + want - 1) / want;
+  kps = (kps + kRouterKTile - 1) / kRouterKTile * kRouterKTile;
+  return static_cast<int>((dm.d + kps - 1) / kps);
+}
+
+static int router_kps(const Dims& dm, int splits) {
+  int kps = (dm.d + splits - 1) / splits;
+  return (kps + kRouterKTile - 1) / kRouterKTile * kRouterKTile;
+}
+
+__global__ void __launch_bounds__(256) router_logits_kernel(const __nv_bfloat16* __restrict__ x,
+                                                            const float* __restrict__ W,
+                                                            float* __restrict__ part, int T,
+                                                            int E, int d, int kps) {
+  __shared__ __align__(16) float Xs[kRouterKTile][kRouterTile + 4];
+  __shared__ __align__(16) float Ws[kRouterKTile][kRouterTile + 4];
+  const int e0 = blockIdx.x * kRouterTile;
+  const int t0 = blockIdx.y * kRouterTile;
+  const int split = blockIdx.z;
+  const int kbeg = split * kps;
+  const int kend = min(d, kbeg + kps);
+  const int tid = threadIdx.x;
+  const int ty = tid >> 4, tx = tid & 15;
+  const int lr = tid >> 2, lc = (tid & 3) * 8;  // loader: row, 8-wide column group
+
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+  for (int k0 = kbeg; k0 < kend; k0 += kRouterKTile) {
+    {
+      const int t = t0 + lr;
+      float v[8];
+      if (t < T) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(x + (size_t)t * d + k0 + lc);
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f2 = __bfloat1622float2(p[i]);
+          v[2 * i] = f2.x;
+          v[2 * i + 1] = f2.y;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) Xs[lc + i][lr] = v[i];
+    }
+    {
+      const int e = e0 + lr;
+      float v[8];
+      if (e < E) {
+        const float4 a = *reinterpret_cast<const float4*>(W + (size_t)e * d + k0 + lc);
+        const float4 b = *reinterpret_cast<const float4*>(W + (size_t)e * d + k0 + lc + 4);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) Ws[lc + i][lr] = v[i];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kRouterKTile; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(&Xs[kk][ty * 4]);
+      const float4 b = *reinterpret_cast<const float4*>(&Ws[kk][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+      const float bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + ty * 4 + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx * 4 + j;
+      if (e < E) part[((size_t)split * T + t) * E + e] = acc[i][j];
+    }
+  }
+}
+
+constexpr int kPerLane = kMaxExperts / 32;
+
+__global__ void __launch_bounds__(256) router_topk_kernel(
+    const float* __restrict__ part, int splits, const float* __restrict__ bias, int T, int E,
+    int k, float scale, int norm, const int32_t* __restrict__ forced, int32_t* __restrict__ ids,
+    float* __restrict__ wts, int32_t* __restrict__ counts, uint32_t* __restrict__ bitmap,
+    int W, uint32_t* __restrict__ status, int32_t* __restrict__ ids_out,
+    float* __restrict__ wts_out) {
+  const int lane = threadIdx.x & 31;
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (t >= T) return;
+  const unsigned full = 0xffffffffu;
+
+  float key[kPerLane], sc[kPerLane];
+#pragma unroll
+  for (int i = 0; i < kPerLane; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E) {
+      float l = 0.f;
+      for (int s = 0; s < splits; ++s) l += part[((size_t)s * T + t) * E + e];
+      const float p = 1.f / (1.f + expf(-l));
+      sc[i] = p;
+      key[i] = p + bias[e];
+    } else {
+      sc[i] = 0.f;
+      key[i] = -INFINITY;
+    }
+  }
+
+  int my_id = 0;
+  float my_sc = 0.f;
+  bool use_forced = forced != nullptr;
+  if (use_forced) {
+    int e = -1;
+    if (lane < k) e = forced[(size_t)t * k + lane];
+    bool bad = lane < k && (e < 0 || e >= E);
+    for (int jj = 0; jj < k; ++jj) {
+      const int other = __shfl_sync(full, e, jj);
+      if (lane < k && jj < lane && other == e) bad = true;
+    }
+    if (__any_sync(full, bad)) {
+      // an out-of-range or repeated id: report it and select normally, which
+      // keeps the dispatch's bookkeeping consistent
+      if (lane == 0) atomicOr(status, MOE_DEVICE_BAD_EXPERT_ID);
+      use_forced = false;
+    } else {
+      // each lane j < k fetches its expert's score from the owning lane
+      for (int jj = 0; jj < k; ++jj) {
+        const int ej = __shfl_sync(full, e, jj);
+        float v = 0.f;
+#pragma unroll
+        for (int i = 0; i < kPerLane; ++i)
+          if (i == (ej >> 5)) v = sc[i];
+        v = __shfl_sync(full, v, ej & 31);
+        if (lane == jj) {
+          my_id = ej;
+          my_sc = v;
+        }
+      }
+    }
+  }
+  if (!use_forced) {
+    uint32_t taken = 0;  // bit i: expert lane + 32 i already chosen
+    for (int j = 0; j < k; ++j) {
+      float bk = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < kPerLane; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && !((taken >> i) & 1u) && (key[i] > bk || (key[i] == bk && e < bi))) {
+          bk = key[i];
+          bi = e;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ok = __shfl_xor_sync(full, bk, off);
+        const int oi = __shfl_xor_sync(full, bi, off);
+        if (ok > bk || (ok == bk && oi < bi)) {
+          bk = ok;
+          bi = oi;
+        }
+      }
+      if (bi >= E) {  // NaN keys: nothing comparable left; keep the bookkeeping valid
+        if (lane == 0) atomicOr(status, MOE_DEVICE_BAD_EXPERT_ID);
+        bi = 0;
+        while (bi < E) {  // smallest id not yet taken
+          const int owner = bi & 31;
+          const uint32_t tk = __shfl_sync(full, taken, owner);
+          if (!((tk >> (bi >> 5)) & 1u)) break;
+          ++bi;
+        }
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      float v = 0.f;
+#pragma unroll
+      for (int i = 0; i < kPerLane; ++i)
+        if (i == (bi >> 5)) v = sc[i];
+      v = __shfl_sync(full, v, bi & 31);
+      if (lane == j) {
+        my_id = bi;
+        my_sc = v;
+      }
+    }
+  }
+
+  float total = lane < k ? my_sc : 0.f;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) total += __shfl_xor_sync(full, total, off);
+  if (lane < k) {
+    const float w = norm ? my_sc / total * scale : my_sc * scale;
+    ids[(size_t)t * k + lane] = my_id;
+    wts[(size_t)t * k + lane] = w;
+    if (ids_out) ids_out[(size_t)t * k + lane] = my_id;
+    if (wts_out) wts_out[(size_t)t * k + lane] = w;
+    atomicAdd(&counts[my_id], 1);
+    atomicOr(&bitmap[(size_t)my_id * W + (t >> 5)], 1u << (t & 31));
+  }
+}
+
+cudaError_t launch_router_logits(moe_handle* h, const void* x, int T, int splits, cudaStream_t s) {
+  const Dims& dm = h->dims;
+  dim3 grid((dm.E + kRouterTile - 1) / kRouterTile, (T + kRouterTile - 1) / kRouterTile, splits);
+  router_logits_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), h->w.router,
+                                            h->ws.logits_part, T, dm.E, dm.d,
+                                            router_kps(dm, splits));
+  h->launches++;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_topk(moe_handle* h, int T, int splits, const int32_t* forced,
+                               cudaStream_t s, int32_t* ids_out, float* wts_out) {
+  const Dims& dm = h->dims;
+  const int W = static_cast<int>((dm.Tmax + 31) / 32);
+  const int blocks = (T * 32 + 255) / 256;
+  router_topk_kernel<<<blocks, 256, 0, s>>>(
+      h->ws.logits_part, splits, h->w.bias, T, dm.E, dm.k, h->cfg.routed_scaling_factor,
+      h->cfg.norm_topk_prob, forced, h->ws.ids, h->ws.wts, h->ws.counts, h->ws.bitmap, W,
+      h->ws.status, ids_out, wts_out);
+  h->launches++;
+  return cudaGetLastError();
+}
+
+}  // namespace smoe

@@ -1,0 +1,199 @@
+"""Parity of the CUDA path with the CPU oracle, through the C ABI.
+
+Tolerances: expert ids bit-exact except near-ties (k-th and (k+1)-th key
+within 1e-5, which may pick either expert but must stay a valid top-k);
+routing weights to 1e-5 relative (fp32 against float64); layer output
+max|gpu - oracle| / max|oracle| <= 1e-2 for BF16 weights (fp32 accumulate,
+BF16 intermediate and output roundings) and <= 3e-2 for FP8.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def smoe():
+    import sparse_moe_sigmoid_b200 as m
+    return m
+
+
+def _check(rep: gu.Report, fmt: str = "bf16"):
+    assert rep.id_mismatch_outside_ties == 0, rep
+    assert rep.invalid_tie_choices == 0, rep
+    assert rep.weight_max_rel < 1e-5, rep
+    assert rep.y_rel_err <= gu.TOL[fmt], rep
+    assert rep.compared_tokens > 0, rep
+
+
+# ------------------------------------------------------------------ tiny layer
+@pytest.fixture(scope="module")
+def tiny(smoe):
+    layer = gu.make_layer(synth.TINY, 300, "bf16")
+    h = gu.create_handle(smoe, layer, max_tokens=300)
+    yield layer, h
+    smoe.moe_destroy(h)
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 17, 64, 129, 300])
+def test_tiny_bf16(smoe, tiny, T):
+    layer, h = tiny
+    x = layer.x[:T].contiguous()
+    y, ids, w = gu.run(smoe, h, layer, x)
+    _check(gu.compare(layer, y, ids, w, x=x))
+
+
+def test_tiny_forced_routing_all_tokens(smoe, tiny):
+    """The oracle's ids fed in: every token's output compares, near-ties too."""
+    layer, h = tiny
+    r = gu.oracle_route(layer)
+    forced = torch.from_numpy(r.ids.astype(np.int32)).cuda()
+    y, ids, w = gu.run(smoe, h, layer, forced=forced)
+    assert np.array_equal(gu.to_np(ids), r.ids)
+    np.testing.assert_allclose(gu.to_np(w), r.weights, rtol=1e-5)
+    yo = gu.oracle_outputs(layer, r.ids, r.weights, np.arange(layer.x.shape[0]))
+    err = np.max(np.abs(gu.to_np(y) - yo)) / np.max(np.abs(yo))
+    assert err <= gu.TOL["bf16"]
+
+
+def test_tiny_weights_sum_and_bias_only_selects(smoe, tiny):
+    layer, h = tiny
+    _, ids, w = gu.run(smoe, h, layer)
+    np.testing.assert_allclose(gu.to_np(w).sum(axis=1), 2.827, rtol=1e-5)
+    assert np.all(gu.to_np(w) > 0)
+    ids = gu.to_np(ids)
+    assert all(len(set(r)) == len(r) for r in ids.tolist())
+
+
+def test_identical_experts_closed_form(smoe):
+    """All routed experts equal to one SwiGLU E and a zero shared expert:
+    y = 2.827 * E(x) whatever the routing."""
+    layer = gu.make_layer(synth.TINY, 96, "bf16", identical=True, shared_zero=True)
+    h = gu.create_handle(smoe, layer, max_tokens=96)
+    try:
+        y, _, _ = gu.run(smoe, h, layer)
+    finally:
+        smoe.moe_destroy(h)
+    m = {n: gu.to_np(v).astype(np.float64) for n, v in synth.expert_slice(layer.ew, 0).items()}
+    from oracle import moe as orc
+    ex = orc.swiglu_expert(gu.to_np(layer.x).astype(np.float64), m["gate"], m["up"], m["down"])
+    err = np.max(np.abs(gu.to_np(y) - 2.827 * ex)) / np.max(np.abs(2.827 * ex))
+    assert err <= gu.TOL["bf16"]
+
+
+def test_two_shared_experts(smoe):
+    """n_shared_experts = 2: the shared MLP has intermediate 2 * f."""
+    shape = synth.LayerShape(hidden_size=256, moe_intermediate_size=128, n_routed_experts=16,
+                             num_experts_per_tok=4, n_shared_experts=2)
+    layer = gu.make_layer(shape, 70, "bf16")
+    h = gu.create_handle(smoe, layer, max_tokens=70)
+    try:
+        y, ids, w = gu.run(smoe, h, layer)
+    finally:
+        smoe.moe_destroy(h)
+    _check(gu.compare(layer, y, ids, w))
+
+
+def test_no_shared_expert(smoe):
+    shape = synth.LayerShape(hidden_size=256, moe_intermediate_size=128, n_routed_experts=16,
+                             num_experts_per_tok=4, n_shared_experts=0)
+    layer = gu.make_layer(shape, 50, "bf16")
+    h = gu.create_handle(smoe, layer, max_tokens=50)
+    try:
+        y, ids, w = gu.run(smoe, h, layer)
+    finally:
+        smoe.moe_destroy(h)
+    _check(gu.compare(layer, y, ids, w))
+
+
+# ------------------------------------------------------------------ edge cases
+def test_edge_cases(smoe, tiny):
+    layer, h = tiny
+    x = layer.x[:8].contiguous()
+    y = torch.full_like(x, 7.0)
+    smoe.moe_forward(h, x, y, T=0, flags=smoe.MOE_FLAG_SYNC_CHECK)  # no-op
+    assert torch.all(y == 7.0)
+    with pytest.raises(smoe.MoeError) as e:
+        big = torch.zeros((301, 256), dtype=torch.bfloat16, device="cuda")
+        smoe.moe_forward(h, big, torch.empty_like(big))
+    assert e.value.status == smoe.MOE_ERR_INVALID_ARG
+    with pytest.raises(smoe.MoeError) as e:
+        smoe.moe_forward(h, x, x)
+    assert e.value.status == smoe.MOE_ERR_INVALID_ARG
+    # a forced id out of range: reported through the status word, the forward
+    # falls back to selecting, and the handle stays usable
+    bad = torch.zeros((8, 4), dtype=torch.int32, device="cuda")
+    bad[3] = torch.tensor([0, 1, 2, 99])
+    with pytest.raises(smoe.MoeError) as e:
+        smoe.moe_forward(h, x, torch.empty_like(x), forced_topk_ids=bad,
+                         flags=smoe.MOE_FLAG_SYNC_CHECK)
+    assert e.value.status == smoe.MOE_ERR_DEVICE
+    assert smoe.moe_get_device_status(h) == 0
+    y2, ids, w = gu.run(smoe, h, layer, x)
+    _check(gu.compare(layer, y2, ids, w, x=x))
+
+
+def test_forward_before_load_is_rejected(smoe):
+    cfg = smoe.moe_config_init_k2(hidden_size=256, moe_intermediate_size=128, n_routed_experts=16,
+                                  num_experts_per_tok=4, max_tokens=4)
+    h = smoe.moe_create(cfg, 0)
+    try:
+        x = torch.zeros((4, 256), dtype=torch.bfloat16, device="cuda")
+        with pytest.raises(smoe.MoeError) as e:
+            smoe.moe_forward(h, x, torch.empty_like(x))
+        assert e.value.status == smoe.MOE_ERR_STATE
+    finally:
+        smoe.moe_destroy(h)
+
+
+def test_host_entry_point_matches_device(smoe, tiny):
+    layer, h = tiny
+    y_dev, _, _ = gu.run(smoe, h, layer)
+    xh = layer.x.cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    smoe.moe_forward_host(h, xh, yh)
+    assert torch.equal(yh, y_dev.cpu())
+
+
+def test_profile_phases(smoe, tiny):
+    layer, h = tiny
+    smoe.moe_profile_enable(h, 3)
+    n0 = smoe.moe_launch_count(h)
+    for _ in range(3):
+        gu.run(smoe, h, layer)
+    ph = smoe.moe_profile_read(h, 3)
+    smoe.moe_profile_enable(h, 0)
+    assert len(ph) == 3 and all(len(p) == smoe.MOE_NUM_PHASES for p in ph)
+    assert all(t >= 0 for p in ph for t in p)
+    assert smoe.moe_launch_count(h) - n0 == 3 * 7
+
+
+# ------------------------------------------------------------------ K2 shapes
+@pytest.fixture(scope="module")
+def k2(smoe):
+    layer = gu.make_layer(synth.K2, 8192, "bf16")
+    h = gu.create_handle(smoe, layer, max_tokens=8192)
+    yield layer, h
+    smoe.moe_destroy(h)
+
+
+def test_k2_decode_T64(smoe, k2):
+    layer, h = k2
+    x = layer.x[:64].contiguous()
+    y, ids, w = gu.run(smoe, h, layer, x)
+    toks = np.random.default_rng(1).choice(64, 6, replace=False)
+    _check(gu.compare(layer, y, ids, w, tokens=toks, x=x))
+
+
+def test_k2_prefill_T8192(smoe, k2):
+    layer, h = k2
+    y, ids, w = gu.run(smoe, h, layer)
+    toks = np.random.default_rng(2).choice(8192, 6, replace=False)
+    rep = gu.compare(layer, y, ids, w, tokens=toks)
+    _check(rep)
+    counts = np.bincount(gu.to_np(ids).ravel(), minlength=384)
+    assert counts.sum() == 8192 * 8 and counts.min() > 0  # ~170 tokens per expert
