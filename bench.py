@@ -1,0 +1,472 @@
+"""Throughput of the K2 routed-MoE layer forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl native|reference]
+
+One step = one forward of the whole layer (router, top-8, dispatch, gate/up
+GEMM + SwiGLU, down GEMM, weighted combine with the shared expert) over one
+batch of T synthetic tokens with weights resident in HBM. Prints one JSON
+line (rank 0).
+
+Workloads (--config):
+  decode      K2 layer, T = 64 tokens, BF16 experts (default)
+  prefill     K2 layer, T = 8192 tokens, BF16 experts
+  fp8-T<n>    K2 layer, T = n tokens, FP8 e4m3 experts with 128x128 scales
+
+N > 1 runs one independent replica per GPU (data parallel over token
+batches; the layer has no exchange step at one GPU per replica), so the
+scaling is weak and the value is the tokens of all ranks / the slowest rank's
+time. Timing: CUDA events on the launch stream, W warm-up steps, then K
+steps between a barrier + synchronize on both sides; max over ranks. The
+weights streamed per step (25-34 GB BF16) are far larger than the 126 MB L2,
+so no flush is needed between steps.
+
+--impl reference times the CPU oracle (float64 numpy) on the host cores, on
+a bounded sample of the same workload each step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "K2 MoE layer tokens/s; % of HBM (decode) / tensor-peak (prefill) roofline"
+UNIT = "tokens/s"
+PHASES = ("router_logits", "router_topk", "route_scan", "dispatch", "gemm_gate_up",
+          "gemm_down", "combine")
+KERNEL_SOURCES = {"gemm_gate_up": ["gemm_bf16.cu", "gemm_fp8.cu", "gemm_common.cuh", "sm100.cuh"],
+                  "gemm_down": ["gemm_bf16.cu", "gemm_fp8.cu", "gemm_common.cuh", "sm100.cuh"]}
+
+
+# ----------------------------------------------------------------- workloads
+def workload(name: str):
+    if name == "decode":
+        return dict(T=64, fmt="bf16", desc="K2 MoE layer decode step, T=64 tokens, BF16 experts")
+    if name == "prefill":
+        return dict(T=8192, fmt="bf16", desc="K2 MoE layer prefill, T=8192 tokens, BF16 experts")
+    if name.startswith("fp8-T"):
+        T = int(name[5:])
+        return dict(T=T, fmt="fp8", desc=f"K2 MoE layer, T={T} tokens, FP8 e4m3 experts "
+                                           "(128x128 block scales, dynamic activation quant)")
+    raise SystemExit(f"unknown --config {name}")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return dict(hbm=j["hbm_gbs"], bf16=j["bf16_tflops"], bf16_sus=j["bf16_tflops_sustained"],
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# ------------------------------------------------------- distributed helpers
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def aggregate_over_ranks(ms: float, tokens: int, device) -> tuple:
+    """(max over ranks of ms, sum over ranks of tokens); identity at world size 1."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return ms, tokens
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    n = torch.tensor([tokens], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(n, op=dist.ReduceOp.SUM)
+    return float(t.item()), int(n.item())
+
+
+def barrier(device):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        t = torch.zeros(1, device=device)
+        dist.all_reduce(t)
+
+
+# ------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+            self.th = threading.Thread(target=self._read, daemon=True)
+            self.th.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.th.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            p = [s.strip() for s in ln.split(",")]
+            if len(p) < 8:
+                continue
+            try:
+                sm.append(float(p[0]))
+                mx = float(p[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, p[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- CPU baseline
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+class OracleSample:
+    """The CPU oracle on a bounded sample of the workload: routing of all T
+    tokens (or of the sample when T is large) and the experts of `n_tok`
+    sampled tokens, with their weights already on the host."""
+
+    def __init__(self, shape, T, fmt, n_tok, x_cpu, Wg_cpu, b_cpu, fetch_expert, seed=7):
+        from oracle import moe as orc
+        self.orc, self.shape, self.fmt = orc, shape, fmt
+        rng = np.random.default_rng(seed)
+        self.T = T
+        self.route_rows = min(T, 256)
+        self.x = x_cpu.float().numpy().astype(np.float64)
+        self.Wg = Wg_cpu.numpy().astype(np.float64)
+        self.b = b_cpu.numpy().astype(np.float64)
+        self.tok = np.sort(rng.choice(T, size=min(n_tok, T), replace=False))
+        rows = np.union1d(self.tok, rng.choice(T, size=self.route_rows, replace=False))
+        self.rows = rows
+        r = orc.route(self.x[rows], self.Wg, self.b, shape.num_experts_per_tok,
+                      shape.routed_scaling_factor, shape.norm_topk_prob)
+        pos = np.searchsorted(rows, self.tok)
+        need = sorted(set(int(e) for e in r.ids[pos].ravel()))
+        self.cache = {e: fetch_expert(e) for e in need}
+        self.shared = fetch_expert(-1) if shape.n_shared_experts > 0 else None
+        self.pos = pos
+
+    def run_once(self) -> int:
+        s, orc = self.shape, self.orc
+        r = orc.route(self.x[self.rows], self.Wg, self.b, s.num_experts_per_tok,
+                      s.routed_scaling_factor, s.norm_topk_prob)
+        orc.experts_combine(self.x[self.rows], r.ids, r.weights, lambda e: self.cache[e],
+                            (lambda: self.shared) if self.shared is not None else None,
+                            self.fmt, s.n_shared_experts, self.pos)
+        return len(self.tok)
+
+    def describe(self):
+        return (f"{len(self.tok)} of {self.T} tokens through the experts (routing for "
+                f"{len(self.rows)} tokens), weights preloaded on the host")
+
+
+def np_expert(mats: dict) -> dict:
+    out = {}
+    for n, v in mats.items():
+        out[n] = v.numpy() if v.dtype == torch.uint8 else v.float().numpy()
+    return out
+
+
+# -------------------------------------------------------------------- arms
+def algorithmic(shape, T, fmt, ids: np.ndarray):
+    """Algorithmic bytes and flops of each GEMM launch for the actual routing."""
+    d, f, E, k, ns = (shape.hidden_size, shape.moe_intermediate_size, shape.n_routed_experts,
+                      shape.num_experts_per_tok, shape.n_shared_experts)
+    wb = 1 if fmt == "fp8" else 2
+    U = len(np.unique(ids))
+    G_used = U + ns
+    R = T * (k + ns)
+    sb = lambda r, c: (r // 128) * (c // 128) * 4 if fmt == "fp8" else 0
+    gate_up_bytes = G_used * 2 * (f * d * wb + sb(f, d)) + R * d * wb + R * f * wb
+    down_bytes = G_used * (d * f * wb + sb(d, f)) + R * f * wb + R * d * 4
+    if fmt == "fp8":
+        gate_up_bytes += R * (d // 128) * 4 + R * (f // 128) * 4
+        down_bytes += R * (f // 128) * 4
+    gate_up_flops = 2 * R * 2 * f * d
+    down_flops = 2 * R * d * f
+    layer_bytes = G_used * 3 * (d * f * wb) + E * d * 4 + E * 4 + T * d * 2 * 2
+    layer_flops = 2 * R * 3 * d * f + 2 * T * E * d
+    return dict(U=U, gemm_gate_up=(gate_up_bytes, gate_up_flops),
+                gemm_down=(down_bytes, down_flops), layer=(layer_bytes, layer_flops))
+
+
+def kernel_src_hash(kernel: str) -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES.get(kernel, []):
+        p = os.path.join(ROOT, "sparse_moe_sigmoid_b200", "csrc", f)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, config: str):
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    j = json.load(open(p)).get(config, {}).get(kernel)
+    if not j or j.get("src") != kernel_src_hash(kernel):
+        return None
+    return j.get("bytes_per_launch")
+
+
+def run_native(args, wl):
+    import sparse_moe_sigmoid_b200 as smoe
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    shape, T, fmt = wl.get("shape", synth.K2), wl["T"], wl["fmt"]
+    x = synth.make_tokens(shape, T, device=dev)
+    Wg, b = synth.make_router(shape, device=dev)
+    ew = synth.make_experts(shape, device=dev, fmt=fmt)
+    cfg = smoe.moe_config_init_k2(
+        max_tokens=T, n_routed_experts=shape.n_routed_experts,
+        weight_format=smoe.MOE_WEIGHT_BF16 if fmt == "bf16" else smoe.MOE_WEIGHT_FP8_E4M3_BLOCK)
+    h = smoe.moe_create(cfg, local)
+    smoe.moe_load_weights(h, Wg, b, ew.gate, ew.up, ew.down, ew.shared_gate, ew.shared_up,
+                          ew.shared_down, ew.gate_scale, ew.up_scale, ew.down_scale,
+                          ew.shared_gate_scale, ew.shared_up_scale, ew.shared_down_scale)
+    y = torch.empty_like(x)
+    ids = torch.empty((T, shape.num_experts_per_tok), dtype=torch.int32, device=dev)
+    smoe.moe_forward(h, x, y, topk_ids_out=ids, flags=smoe.MOE_FLAG_SYNC_CHECK)
+    ids_np = ids.cpu().numpy()
+
+    # CPU oracle baseline (rank 0, one GPU only), before the caller copies go
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        n_tok = 4 if T <= 64 else 3
+        ors = OracleSample(shape, T, fmt, n_tok, x.cpu(), Wg.cpu(), b.cpu(),
+                           lambda e: np_expert(synth.expert_slice(ew, e) if e >= 0
+                                               else synth.shared_slice(ew)))
+        t0 = time.perf_counter()
+        n, reps = 0, 0
+        while True:
+            n += ors.run_once()
+            reps += 1
+            if time.perf_counter() - t0 > 10.0 or reps >= 20:
+                break
+        el = time.perf_counter() - t0
+        cpu = {"value": n / el, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{ors.describe()}; {reps} repetitions in {el:.1f} s"}
+    del ew
+    torch.cuda.empty_cache()
+
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        smoe.moe_forward(h, x, y)
+    torch.cuda.synchronize()
+
+    smoe.moe_profile_enable(h, args.steps)
+    n0 = smoe.moe_launch_count(h)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(dev)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        smoe.moe_forward(h, x, y)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(dev)
+    clk = clocks.stop()
+    launches = smoe.moe_launch_count(h) - n0
+    ms_total = e0.elapsed_time(e1)
+    phases = np.array(smoe.moe_profile_read(h, args.steps))
+    smoe.moe_profile_enable(h, 0)
+    st = smoe.moe_get_device_status(h)
+    if st:
+        raise SystemExit(f"device status word set during the timed steps: {st:#x}")
+
+    # end to end through the host-memory entry point, copies included
+    xh = x.cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    for _ in range(2):
+        smoe.moe_forward_host(h, xh, yh)
+    n_e2e = max(3, min(args.steps, 50))
+    barrier(dev)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(n_e2e):
+        smoe.moe_forward_host(h, xh, yh)  # copies in, forward, copy out, synchronise
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
+    e2e_ms, _ = aggregate_over_ranks(e2e_ms, T, dev)
+
+    ms_step = ms_total / args.steps
+    ms_max, tokens_all = aggregate_over_ranks(ms_step, T, dev)
+    value = tokens_all / (ms_max / 1e3)
+
+    # roofline of the dominant kernel, timed live by the library's phase events
+    mean_ph = phases.mean(axis=0)
+    dom = int(np.argmax(mean_ph))
+    dom_name = PHASES[dom]
+    alg = algorithmic(shape, T, fmt, ids_np)
+    peaks = load_peaks()
+    byts, flops = alg.get(dom_name, alg["layer"])
+    dur = mean_ph[dom] / 1e3
+    hbm_t = byts / (peaks["hbm"] * 1e9)
+    ten_t = flops / (peaks["bf16_sus"] * 1e12 * (2.0 if fmt == "fp8" else 1.0))
+    if hbm_t >= ten_t:
+        roof = {"bound": "hbm", "achieved": byts / dur / 1e9, "peak": peaks["hbm"],
+                "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": flops / dur / 1e12,
+                "peak": peaks["bf16_sus"] * (2.0 if fmt == "fp8" else 1.0), "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = traffic_for(dom_name, args.config)
+    roof.update({
+        "kernel": dom_name, "launch_ms": round(mean_ph[dom], 4),
+        "algorithmic_bytes": int(byts), "algorithmic_flops": int(flops),
+        "hbm_frac": (byts / dur / 1e9) / peaks["hbm"],
+        "tensor_frac": (flops / dur / 1e12) / (peaks["bf16_sus"] * (2.0 if fmt == "fp8" else 1.0)),
+        "peak_source": f"{peaks['src']} (HBM copy GB/s; sustained cuBLAS bf16 TF/s"
+                       f"{', x2 nominal fp8 ratio' if fmt == 'fp8' else ''})"})
+    layer_bytes, layer_flops = alg["layer"]
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if fmt == "bf16" else "e4m3",
+        "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) weights, random init)",
+        "config": {"workload": wl["desc"], "tokens": T, "global_batch": T * ws,
+                   "hidden_size": shape.hidden_size, "n_routed_experts": shape.n_routed_experts,
+                   "top_k": shape.num_experts_per_tok, "moe_intermediate_size":
+                       shape.moe_intermediate_size, "parallelism": f"replicas x{ws}",
+                   "distinct_experts_hit": alg["U"],
+                   "l2": "no flush: the expert weights streamed each step exceed the 126 MB L2"},
+        "roofline": roof,
+        "layer_roofline": {"bytes": int(layer_bytes), "flops": int(layer_flops),
+                           "hbm_frac": (layer_bytes / (ms_max / 1e3) / 1e9) / peaks["hbm"]},
+        "phases_ms": {p: round(float(v), 4) for p, v in zip(PHASES, mean_ph)},
+        "cpu_baseline": cpu,
+        "e2e": {"value": tokens_all / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 2),
+                "ms_per_step": e2e_ms, "api": "moe_forward_host (pinned host x and y)"},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    smoe.moe_destroy(h)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def run_reference(args, wl):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    shape, T, fmt = wl.get("shape", synth.K2), wl["T"], wl["fmt"]
+    x = synth.make_tokens(shape, T)
+    Wg, b = synth.make_router(shape)
+    n_tok = 2
+    ors = OracleSample(shape, T, fmt, n_tok, x, Wg, b,
+                       lambda e: np_expert(synth.make_expert(shape, e, fmt=fmt)))
+    for _ in range(args.warmup):
+        ors.run_once()
+    t0 = time.perf_counter()
+    n = 0
+    for _ in range(args.steps):
+        n += ors.run_once()
+    el = time.perf_counter() - t0
+    value = n / el
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "impl": "reference",
+        "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) weights, random init)",
+        "config": {"workload": wl["desc"], "tokens": T, "global_batch": T * ws,
+                   "hidden_size": shape.hidden_size, "n_routed_experts": shape.n_routed_experts,
+                   "top_k": shape.num_experts_per_tok,
+                   "moe_intermediate_size": shape.moe_intermediate_size,
+                   "parallelism": "host cores, rank 0 only"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"each step: {ors.describe()}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="decode")
+    ap.add_argument("--impl", default="native", choices=("native", "reference"))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override T (small profiling cases)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override n_routed_experts (small profiling cases)")
+    args = ap.parse_args(argv)
+    wl = workload(args.config)
+    if args.tokens is not None or args.experts is not None:
+        wl["T"] = args.tokens or wl["T"]
+        E = args.experts or synth.K2.n_routed_experts
+        wl["shape"] = synth.LayerShape(n_routed_experts=E)
+        wl["desc"] += f" [reduced case: T={wl['T']}, {E} routed experts]"
+    if args.steps is None:
+        args.steps = (400 if wl["T"] <= 1024 else 100) if args.impl == "native" else 5
+    if args.warmup < 3 and args.impl == "native":
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_native(args, wl)
+
+
+if __name__ == "__main__":
+    main()

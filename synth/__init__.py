@@ -212,3 +212,23 @@ def shared_slice(ew: ExpertWeights):
         out.update(gate_scale=ew.shared_gate_scale.cpu(), up_scale=ew.shared_up_scale.cpu(),
                    down_scale=ew.shared_down_scale.cpu())
     return out
+
+
+def make_expert(shape: LayerShape, e: int, seed: int = SEED, device="cpu", fmt: str = "bf16"):
+    """One routed expert's matrices alone (e < E), or the shared expert (e = -1),
+    drawn exactly as make_experts draws them on the same device type.
+    Returns {"gate", "up", "down"} (+ "*_scale" for FP8)."""
+    d, f = shape.hidden_size, shape.moe_intermediate_size
+    out = {}
+    for n, rc in (("gate", (f, d)), ("up", (f, d)), ("down", (d, f))):
+        if e < 0:
+            fs = f * shape.n_shared_experts
+            rc = (fs, d) if n != "down" else (d, fs)
+            w = _expert_matrix(rc, seed, "shared_" + n, 0, device)
+        else:
+            w = _expert_matrix(rc, seed, n, e, device)
+        if fmt == "bf16":
+            out[n] = w.to(torch.bfloat16)
+        else:
+            out[n], out[n + "_scale"] = quantize_blocks_e4m3(w)
+    return out

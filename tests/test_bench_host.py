@@ -1,0 +1,71 @@
+"""Host logic of bench.py without a GPU: the multi-rank aggregation (max of
+the per-rank step time, sum of tokens) over a 2-rank gloo group, the
+workload table, and the algorithmic byte/flop counts."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+import synth
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, ws, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(ws))
+    dist.init_process_group("gloo", rank=rank, world_size=ws)
+    try:
+        ms, tok = bench.aggregate_over_ranks(1.0 + rank * 2.5, 64, torch.device("cpu"))
+        bench.barrier(torch.device("cpu"))
+        out[rank] = (ms, tok)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_aggregate_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        port = _free_port()
+        mp.start_processes(_worker, args=(2, port, out), nprocs=2, join=True,
+                           start_method="spawn")
+        res = dict(out)
+    assert res[0] == res[1] == (3.5, 128)
+
+
+def test_single_rank_is_identity():
+    assert bench.aggregate_over_ranks(2.0, 64, torch.device("cpu")) == (2.0, 64)
+
+
+def test_workloads():
+    assert bench.workload("decode")["T"] == 64
+    assert bench.workload("prefill")["T"] == 8192
+    w = bench.workload("fp8-T1024")
+    assert w["T"] == 1024 and w["fmt"] == "fp8"
+    with pytest.raises(SystemExit):
+        bench.workload("nope")
+
+
+def test_algorithmic_counts_match_the_expert_size():
+    # every expert hit once: the weight bytes are (E + 1) experts x 3 matrices
+    s = synth.K2
+    ids = np.arange(384).reshape(48, 8)
+    a = bench.algorithmic(s, 48, "bf16", ids)
+    assert a["U"] == 384
+    per_expert = 3 * 7168 * 2048 * 2  # BF16: 88,080,384 bytes per expert
+    assert per_expert == 88080384
+    assert a["layer"][0] - (385 * per_expert) == 384 * 7168 * 4 + 384 * 4 + 48 * 7168 * 4
+    R = 48 * 9
+    assert a["gemm_gate_up"][1] == 2 * R * 2 * 2048 * 7168
