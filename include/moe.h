@@ -178,6 +178,41 @@ moe_status_t moe_profile_read(moe_handle_t* h, float* ms, int32_t cap, int32_t* 
 /* Number of kernels this handle has launched so far. */
 int64_t moe_launch_count(const moe_handle_t* h);
 
+/* Router alone, with no device allocation of any kind (no handle).
+ *
+ * The pages have no counterpart of this call; it exists for callers that
+ * cannot call cudaMalloc: engines that hand nearly all GPU memory to their
+ * own pool at start-up, and latency-critical steps that cannot afford the
+ * device synchronisation cudaMalloc may cause. It computes what moe_forward
+ * computes for routing (the same kernels): for T tokens, the
+ * num_experts_per_tok experts with the largest sigmoid score + bias, key
+ * descending, and their weights (unbiased scores, normalised when
+ * norm_topk_prob = 1, times routed_scaling_factor).
+ *
+ *   x              device BF16 [T, hidden_size], 16-byte aligned
+ *   router_weight  device fp32 [n_routed_experts, hidden_size], 16-byte aligned
+ *   e_score_correction_bias  device fp32 [n_routed_experts]
+ *   topk_ids       device int32 [T, num_experts_per_tok] (written)
+ *   topk_weights   device fp32 [T, num_experts_per_tok] (written)
+ *   stream         cudaStream_t as void*; the call is asynchronous on it
+ *
+ * Runs on the calling thread's current device. Scratch lives in a 16 MiB
+ * device array inside the library, one per GPU, kept until the process
+ * exits. A call needs 4 * (T * n_routed_experts + n_routed_experts *
+ * (1 + ceil(T / 32))) + 512 bytes of it at the least; bigger T returns
+ * MOE_ERR_INVALID_ARG (for 384 experts, T up to about 10,600). The first call
+ * on each device looks up the array's device address (cudaGetSymbolAddress);
+ * make that first call before any stream capture. Every call reuses the same
+ * array: calls whose GPU work can overlap (unordered streams, several host
+ * threads) race and must not be made. hidden_size must be a multiple of 32,
+ * n_routed_experts <= 512, num_experts_per_tok <= 32 (else
+ * MOE_ERR_UNSUPPORTED). */
+moe_status_t moe_router_topk_noalloc(const void* x, int64_t T, const float* router_weight,
+                                     const float* e_score_correction_bias, int32_t hidden_size,
+                                     int32_t n_routed_experts, int32_t num_experts_per_tok,
+                                     int32_t norm_topk_prob, float routed_scaling_factor,
+                                     int32_t* topk_ids, float* topk_weights, void* stream);
+
 /* Free everything the handle owns. NULL is a no-op. Synchronises the device. */
 void moe_destroy(moe_handle_t* h);
 

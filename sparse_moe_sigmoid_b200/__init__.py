@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libsmoe_b200.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m sparse_moe_sigmoid_b200.build`")
+        f"{LIB_PATH} is missing: build it with `python sparse_moe_sigmoid_b200/build.py`")
 _lib = ctypes.CDLL(LIB_PATH)
 
 # ---------------------------------------------------------------- constants
@@ -79,6 +79,10 @@ _sig = {
     "moe_profile_enable": (_S, [_H, ctypes.c_int32]),
     "moe_profile_read": (_S, [_H, ctypes.POINTER(ctypes.c_float), ctypes.c_int32,
                               ctypes.POINTER(ctypes.c_int32)]),
+    "moe_router_topk_noalloc": (_S, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                     ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
+                                     ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
+                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "moe_launch_count": (ctypes.c_int64, [_H]),
     "moe_destroy": (None, [_H]),
     "moe_status_string": (ctypes.c_char_p, [_S]),
@@ -201,6 +205,20 @@ def moe_profile_read(h, max_forwards: int):
     _check(_lib.moe_profile_read(h, buf, cap, ctypes.byref(n)), "moe_profile_read", h)
     n = min(n.value, max_forwards)
     return [[buf[i * MOE_NUM_PHASES + p] for p in range(MOE_NUM_PHASES)] for i in range(n)]
+
+
+def moe_router_topk_noalloc(x, router_weight, e_score_correction_bias, num_experts_per_tok: int,
+                            topk_ids, topk_weights, norm_topk_prob: int = 1,
+                            routed_scaling_factor: float = 2.827, T: Optional[int] = None,
+                            stream=None):
+    """Routing only, with the library's static scratch (no allocation)."""
+    T = x.shape[0] if T is None else T
+    E, d = router_weight.shape
+    st = _lib.moe_router_topk_noalloc(_ptr(x), T, _ptr(router_weight),
+                                      _ptr(e_score_correction_bias), d, E, num_experts_per_tok,
+                                      norm_topk_prob, routed_scaling_factor, _ptr(topk_ids),
+                                      _ptr(topk_weights), _stream(stream))
+    _check(st, "moe_router_topk_noalloc")
 
 
 def moe_launch_count(h) -> int:

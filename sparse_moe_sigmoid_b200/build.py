@@ -2,7 +2,8 @@
 
 Compiles every csrc/*.cu to an object in parallel, then links one shared
 library into this package directory. Needs nvcc but no GPU.
-Usage: python -m sparse_moe_sigmoid_b200.build [--verbose]
+Usage: python sparse_moe_sigmoid_b200/build.py [--verbose]
+(run it as a file: importing the package first would load the old library)
 """
 from __future__ import annotations
 

@@ -94,6 +94,10 @@ int router_splits(const Dims& dm, int64_t T, int num_sms);
 cudaError_t launch_router_logits(moe_handle* h, const void* x, int T, int splits, cudaStream_t s);
 cudaError_t launch_router_topk(moe_handle* h, int T, int splits, const int32_t* forced,
                                cudaStream_t s, int32_t* ids_out, float* wts_out);
+cudaError_t launch_router_raw(const void* x, const float* router_weight, const float* bias, int T,
+                              int d, int E, int k, float scale, int norm, int splits, float* part,
+                              int32_t* counts, uint32_t* bitmap, int W, uint32_t* status,
+                              int32_t* ids, float* wts, cudaStream_t s);
 // dispatch.cu
 GemmPlan plan_gate_up(const Dims& dm, int64_t T);
 GemmPlan plan_down(const Dims& dm, int64_t T);

@@ -269,4 +269,24 @@ cudaError_t launch_router_topk(moe_handle* h, int T, int splits, const int32_t* 
   return cudaGetLastError();
 }
 
+// Both router kernels on caller-supplied buffers (no handle): used by the
+// entry point that keeps its scratch in a static device array.
+cudaError_t launch_router_raw(const void* x, const float* router_weight, const float* bias, int T,
+                              int d, int E, int k, float scale, int norm, int splits, float* part,
+                              int32_t* counts, uint32_t* bitmap, int W, uint32_t* status,
+                              int32_t* ids, float* wts, cudaStream_t s) {
+  Dims dm{};
+  dm.d = d;
+  dm.E = E;
+  dim3 grid((E + kRouterTile - 1) / kRouterTile, (T + kRouterTile - 1) / kRouterTile, splits);
+  router_logits_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), router_weight,
+                                            part, T, E, d, router_kps(dm, splits));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int blocks = (T * 32 + 255) / 256;
+  router_topk_kernel<<<blocks, 256, 0, s>>>(part, splits, bias, T, E, k, scale, norm, nullptr, ids,
+                                            wts, counts, bitmap, W, status, nullptr, nullptr);
+  return cudaGetLastError();
+}
+
 }  // namespace smoe
