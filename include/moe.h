@@ -175,6 +175,19 @@ moe_status_t moe_get_device_status(moe_handle_t* h, uint32_t* flags);
 moe_status_t moe_profile_enable(moe_handle_t* h, int32_t max_forwards);
 moe_status_t moe_profile_read(moe_handle_t* h, float* ms, int32_t cap, int32_t* n_forwards);
 
+/* The FP8 path's dynamic activation quantisation on its own: for each of
+ * `rows` rows of x (device BF16 [rows, cols], cols a multiple of 128), and
+ * each 128-column group, s = amax/448 (amax = 0 -> s = 1) and
+ * q = e4m3(v / s), both divisions correctly rounded, the conversion
+ * nearest-even and saturating at 448 (config.json quantization_config:
+ * activation_scheme dynamic, fmt e4m3, on the "Kimi K2 · Down projection"
+ * page; the per-128-column granularity is this library's reading).
+ * Writes q (device uint8 [rows, cols]) and scales (device fp32
+ * [rows, cols/128]). x and q 16-byte aligned. Runs on the current device,
+ * asynchronous on `stream`. This is the kernel moe_forward applies to x. */
+moe_status_t moe_act_quant_e4m3(const void* x, int64_t rows, int32_t cols, void* q,
+                                float* scales, void* stream);
+
 /* Number of kernels this handle has launched so far. */
 int64_t moe_launch_count(const moe_handle_t* h);
 

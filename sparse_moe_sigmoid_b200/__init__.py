@@ -83,6 +83,8 @@ _sig = {
                                      ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
                                      ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "moe_act_quant_e4m3": (_S, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p,
+                                ctypes.c_void_p, ctypes.c_void_p]),
     "moe_launch_count": (ctypes.c_int64, [_H]),
     "moe_destroy": (None, [_H]),
     "moe_status_string": (ctypes.c_char_p, [_S]),
@@ -219,6 +221,13 @@ def moe_router_topk_noalloc(x, router_weight, e_score_correction_bias, num_exper
                                       norm_topk_prob, routed_scaling_factor, _ptr(topk_ids),
                                       _ptr(topk_weights), _stream(stream))
     _check(st, "moe_router_topk_noalloc")
+
+
+def moe_act_quant_e4m3(x, q, scales, stream=None):
+    """Per-row, per-128-column e4m3 quantisation of a BF16 [rows, cols] tensor."""
+    rows, cols = x.shape
+    st = _lib.moe_act_quant_e4m3(_ptr(x), rows, cols, _ptr(q), _ptr(scales), _stream(stream))
+    _check(st, "moe_act_quant_e4m3")
 
 
 def moe_launch_count(h) -> int:

@@ -145,6 +145,9 @@ moe_status_t validate(const moe_config_t* c, std::string* why) {
   if (c->weight_format == MOE_WEIGHT_FP8_E4M3_BLOCK &&
       c->activation_scheme != MOE_ACTIVATION_DYNAMIC)
     return unsup("FP8 needs activation_scheme dynamic");
+  if (c->weight_format == MOE_WEIGHT_FP8_E4M3_BLOCK &&
+      (c->hidden_size > 8192 || c->moe_intermediate_size > 8192))
+    return unsup("FP8: hidden_size and moe_intermediate_size <= 8192");
   const int64_t rows = c->max_tokens * (c->num_experts_per_tok + c->n_shared_experts);
   if (c->max_tokens > (1 << 20) || rows > (int64_t(1) << 30))
     return unsup("max_tokens too large (at most 2^20 tokens)");
@@ -539,6 +542,19 @@ moe_status_t moe_profile_read(moe_handle_t* h, float* ms, int32_t cap, int32_t* 
     }
   }
   return MOE_OK;
+}
+
+moe_status_t moe_act_quant_e4m3(const void* x, int64_t rows, int32_t cols, void* q, float* scales,
+                                void* stream) {
+  if (rows < 0 || cols <= 0 || cols % 128 != 0) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (x == nullptr || q == nullptr || scales == nullptr) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(q)) & 15)
+    return MOE_ERR_INVALID_ARG;
+  if (rows > (int64_t(1) << 26)) return MOE_ERR_INVALID_ARG;
+  cudaError_t e = smoe::launch_act_quant(x, rows, cols, static_cast<uint8_t*>(q), scales,
+                                         static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int64_t moe_launch_count(const moe_handle_t* h) { return h ? h->launches : 0; }

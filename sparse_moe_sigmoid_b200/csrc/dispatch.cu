@@ -166,23 +166,12 @@ __global__ void __launch_bounds__(256) dispatch_bf16_kernel(
   for (int c = lane; c < n16; c += 32) dst[c] = __ldg(src + c);
 }
 
-__global__ void __launch_bounds__(256) dispatch_fp8_kernel(
-    const __nv_bfloat16* __restrict__ x, int T, int d, int k, int E, int items,
-    const int32_t* __restrict__ ids, const uint32_t* __restrict__ bitmap,
-    const int32_t* __restrict__ word_prefix, const int32_t* __restrict__ offsets, int W,
-    int32_t* __restrict__ pair_row, int32_t* __restrict__ row_token, uint8_t* __restrict__ xq,
-    float* __restrict__ xs) {
-  const int lane = threadIdx.x & 31;
-  const int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (i >= items) return;
-  int t;
-  const int row = place_row(i, T, k, E, ids, bitmap, word_prefix, offsets, W, &t);
-  if (lane == 0) {
-    if (i < T * k) pair_row[i] = row;
-    row_token[row] = t;
-  }
+// One row of d BF16 values -> d e4m3 codes + d/128 fp32 scales, by one warp:
+// each half-warp takes one 128-column group (16 lanes x 8 values).
+__device__ __forceinline__ void quant_row_e4m3(const __nv_bfloat16* __restrict__ src, int d,
+                                               uint8_t* __restrict__ dst,
+                                               float* __restrict__ scales, int lane) {
   const int ngroups = d / 128;
-  // each half-warp quantises one 128-column group: 16 lanes x 8 values
   for (int g0 = 0; g0 < ngroups; g0 += 2) {
     const int gi = g0 + (lane >> 4);
     const bool active = gi < ngroups;
@@ -190,7 +179,7 @@ __global__ void __launch_bounds__(256) dispatch_fp8_kernel(
     float v[8];
     float amax = 0.f;
     if (active) {
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d + col));
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src + col));
       const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -216,10 +205,47 @@ __global__ void __launch_bounds__(256) dispatch_fp8_kernel(
         if (j & 1) packed[j >> 1] |= static_cast<uint32_t>(b) << 16;
         else packed[j >> 1] = static_cast<uint32_t>(b);
       }
-      *reinterpret_cast<uint2*>(xq + (size_t)row * d + col) = make_uint2(packed[0], packed[1]);
-      if ((lane & 15) == 0) xs[(size_t)row * ngroups + gi] = sa;
+      *reinterpret_cast<uint2*>(dst + col) = make_uint2(packed[0], packed[1]);
+      if ((lane & 15) == 0) scales[gi] = sa;
     }
   }
+}
+
+__global__ void __launch_bounds__(256) dispatch_fp8_kernel(
+    const __nv_bfloat16* __restrict__ x, int T, int d, int k, int E, int items,
+    const int32_t* __restrict__ ids, const uint32_t* __restrict__ bitmap,
+    const int32_t* __restrict__ word_prefix, const int32_t* __restrict__ offsets, int W,
+    int32_t* __restrict__ pair_row, int32_t* __restrict__ row_token, uint8_t* __restrict__ xq,
+    float* __restrict__ xs) {
+  const int lane = threadIdx.x & 31;
+  const int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (i >= items) return;
+  int t;
+  const int row = place_row(i, T, k, E, ids, bitmap, word_prefix, offsets, W, &t);
+  if (lane == 0) {
+    if (i < T * k) pair_row[i] = row;
+    row_token[row] = t;
+  }
+  quant_row_e4m3(x + (size_t)t * d, d, xq + (size_t)row * d, xs + (size_t)row * (d / 128), lane);
+}
+
+// Dynamic activation quantisation of a dense [rows, d] BF16 matrix.
+__global__ void __launch_bounds__(256) act_quant_kernel(const __nv_bfloat16* __restrict__ x,
+                                                        int64_t rows, int d,
+                                                        uint8_t* __restrict__ q,
+                                                        float* __restrict__ s) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (r >= rows) return;
+  quant_row_e4m3(x + r * d, d, q + r * d, s + r * (d / 128), lane);
+}
+
+cudaError_t launch_act_quant(const void* x, int64_t rows, int d, uint8_t* q, float* s,
+                             cudaStream_t st) {
+  const int64_t blocks = (rows * 32 + 255) / 256;
+  act_quant_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(x), rows, d, q, s);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_dispatch(moe_handle* h, const void* x, int T, cudaStream_t s) {

@@ -1,11 +1,369 @@
-// Grouped expert GEMMs for e4m3 weights with 128x128 block scales.
+// Grouped expert GEMMs for e4m3 weights with one fp32 scale per 128x128 block
+// and dynamically quantised e4m3 activations (one fp32 scale per row per 128
+// columns).
+//
+// Weight format: "Kimi K2 · Down projection" (OpenModelAtlas), the
+// config.json quantization_config excerpt (fmt e4m3, weight_block_size
+// [128, 128], activation_scheme dynamic) and the note that every 128 x 128
+// block carries one scale. With W = q_w * s_w and x = q_x * s_x per block,
+//   (W x)[n] = sum_kb  s_w[n/128, kb] * s_x[kb] * sum_{k in kb} q_w[n,k] q_x[k]
+// The inner sum is an e4m3 x e4m3 tensor-core MMA (tcgen05 kind::f8f6f4,
+// K = 32 per instruction, 4 per 128-column block) into an fp32 partial in
+// TMEM; the scales differ per block, so each block's partial is promoted
+// separately: four promotion warps read it (tcgen05.ld), multiply by
+// s_w * s_x[row] and add into fp32 registers. The partial lives in two TMEM
+// buffers used in turn, so the MMAs of block kb+1 run while block kb is
+// promoted. (The hardware's own block scaling takes power-of-two ue8m0
+// scales per 32 columns; the K2 scales are arbitrary fp32 per 128, so it does
+// not apply.)
+//
+// Gate/up epilogue: h = silu(g) * u in fp32, then h is quantised per row per
+// 128 features, which is exactly this tile's 128 features: s_h = amax/448,
+// q = e4m3(h / s_h) (correctly rounded divisions, nearest-even saturating
+// conversion), written with its scale for the down GEMM.
+// Down epilogue: the promoted fp32 row outputs.
+//
+// Roles and the bounded-wait / wind-down rules are those of the BF16 kernel
+// (gemm_bf16.cu): warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
+// warps 2..5 promotion + epilogue.
+#include <cuda_fp8.h>
+
+#include "gemm_common.cuh"
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace smoe {
 
+using namespace sm100;
+
+constexpr int kFp8MaxKBlocks = 64;  // hidden_size and moe_intermediate_size <= 8192
+
+template <int BN, bool GATED>
+struct Fp8Cfg {
+  static constexpr int kA = 128 * 128;  // 128 rows x 128 e4m3
+  static constexpr int kB = BN * 128;
+  static constexpr int kNumA = GATED ? 2 : 1;
+  static constexpr int kStage = kA * kNumA + kB;
+  static constexpr int kScaleBytes = (kFp8MaxKBlocks * BN + 2 * kFp8MaxKBlocks) * 4;
+  static constexpr int kAmaxBytes = 4 * BN * 4;
+  static constexpr int kStages0 = (227 * 1024 - 2048 - kScaleBytes - kAmaxBytes) / kStage;
+  static constexpr int kStages = kStages0 > 10 ? 10 : kStages0;
+  static constexpr int kPCols = GATED ? 2 * BN : BN;  // one partial buffer
+  static constexpr int kTmemCols = pow2_at_least(2 * kPCols, 32);
+  static constexpr int kSmem = kStages * kStage + kScaleBytes + kAmaxBytes + 1024 + 320;
+  static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
+  static_assert(kStages >= 2, "need at least two stages");
+};
+
+template <int BN, bool GATED>
+__global__ void __launch_bounds__(192, 1)
+    grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA0,
+                            const __grid_constant__ CUtensorMap tmA1,
+                            const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+  using C = Fp8Cfg<BN, GATED>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  float* sa_s = reinterpret_cast<float*>(smem + C::kStages * C::kStage);  // [KB][BN]
+  float* sw_s = sa_s + kFp8MaxKBlocks * BN;                                // [2][KB]
+  float* amax_s = sw_s + 2 * kFp8MaxKBlocks;                               // [4][BN]
+  uint64_t* full = reinterpret_cast<uint64_t*>(amax_s + 4 * BN);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* pfull = empty + C::kStages;
+  uint64_t* pempty = pfull + 2;
+  uint64_t* drain = pempty + 2;
+  uint64_t* grp = drain + 1;  // the 128 promotion threads' own barrier (bounded waits)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(grp + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  volatile uint32_t* consumed = tmem_slot + 2;
+  volatile uint32_t* issued = tmem_slot + 3;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int KB = args.k_blocks;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&pfull[a], 1);
+      mbar_init(&pempty[a], 4);
+    }
+    mbar_init(drain, 1);
+    mbar_init(grp, 128);
+    *abort_flag = 0;
+    *consumed = 0;
+    *issued = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA0);
+    if (GATED) tma_prefetch_desc(&tmA1);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total_units = __ldg(args.unit_base + args.G);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+        const Unit un = decode_unit(u, args, BN);
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % C::kStages;
+          const uint32_t ph = (it / C::kStages) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * C::kStage;
+          mbar_arrive_expect_tx(&full[s], C::kStage);
+          tma_load_3d(st, &tmA0, &full[s], kb * 128, un.mt * 128, un.g);
+          if (GATED) tma_load_3d(st + C::kA, &tmA1, &full[s], kb * 128, un.mt * 128, un.g);
+          tma_load_2d(st + C::kA * C::kNumA, &tmB, &full[s], kb * 128, un.row0);
+          *issued = it + 1;
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(args.status, MOE_DEVICE_WAIT_TIMEOUT);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      uint32_t it = 0;  // k-blocks issued so far (also the partial-buffer sequence)
+      bool ok = true;
+      for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+        const Unit un = decode_unit(u, args, BN);
+        const uint32_t n = static_cast<uint32_t>(((un.nvalid + 15) / 16) * 16);
+        const uint32_t idesc = make_idesc(0u, n);
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % C::kStages;
+          const uint32_t ph = (it / C::kStages) & 1u;
+          const int pb = it & 1;
+          if (!mbar_wait(&pempty[pb], ((it >> 1) & 1u) ^ 1u, abort_flag) ||
+              !mbar_wait(&full[s], ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + s * C::kStage);
+          const uint64_t ad0 = sw128_kmajor_desc(a0);
+          const uint64_t ad1 = sw128_kmajor_desc(a0 + C::kA);
+          const uint64_t bd = sw128_kmajor_desc(a0 + C::kA * C::kNumA);
+          const uint32_t d0 = tmem_base + pb * C::kPCols;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t accum = k ? 1u : 0u;  // each block's partial starts fresh
+            mma_fp8(d0, ad0 + 2 * k, bd + 2 * k, idesc, accum);
+            if (GATED) mma_fp8(d0 + BN, ad1 + 2 * k, bd + 2 * k, idesc, accum);
+          }
+          mma_commit(&empty[s]);
+          mma_commit(&pfull[pb]);
+          *consumed = it + 1;
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(args.status, MOE_DEVICE_WAIT_TIMEOUT);
+      }
+      mma_commit(drain);
+      mbar_wait(drain, 0, nullptr);
+    }
+  } else {
+    const int q = warp & 3;           // TMEM lane quarter
+    const int ptid = threadIdx.x - 64;  // 0..127 among the promotion warps
+    uint32_t it = 0, gph = 0;
+    bool ok = true;
+    auto group_sync = [&]() {
+      mbar_arrive(grp);
+      const bool r = mbar_wait(grp, gph, abort_flag);
+      gph ^= 1u;
+      return r;
+    };
+    for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+      const Unit un = decode_unit(u, args, BN);
+      // this tile's scales: activations [KB][BN] and the weight block scales
+      if (!group_sync()) {  // the previous tile's readers are done
+        ok = false;
+        break;
+      }
+      for (int i = ptid; i < KB * BN; i += 128) {
+        const int kb = i / BN, j = i - kb * BN;
+        sa_s[i] = j < un.nvalid ? __ldg(args.act_scale + (size_t)(un.row0 + j) * KB + kb) : 0.f;
+      }
+      const size_t wrow = ((size_t)un.g * args.m_tiles + un.mt) * KB;
+      for (int i = ptid; i < KB; i += 128) {
+        sw_s[i] = __ldg(args.w_scale0 + wrow + i);
+        if (GATED) sw_s[kFp8MaxKBlocks + i] = __ldg(args.w_scale1 + wrow + i);
+      }
+      if (!group_sync()) {
+        ok = false;
+        break;
+      }
+
+      float acc0[BN], acc1[GATED ? BN : 1];
+#pragma unroll
+      for (int j = 0; j < BN; ++j) {
+        acc0[j] = 0.f;
+        if (GATED) acc1[j] = 0.f;
+      }
+      const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const int pb = it & 1;
+        if (!mbar_wait(&pfull[pb], (it >> 1) & 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float sw0 = sw_s[kb];
+        const float sw1 = GATED ? sw_s[kFp8MaxKBlocks + kb] : 0.f;
+        const float* sa = sa_s + kb * BN;
+#pragma unroll
+        for (int c = 0; c < BN / 16; ++c) {
+          if (c * 16 < un.nvalid) {
+            uint32_t g[16], v[16];
+            tmem_ld16(tq + pb * C::kPCols + c * 16, g);
+            if (GATED) tmem_ld16(tq + pb * C::kPCols + BN + c * 16, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float s = sa[c * 16 + j];
+              acc0[c * 16 + j] = fmaf(__uint_as_float(g[j]), sw0 * s, acc0[c * 16 + j]);
+              if (GATED) acc1[c * 16 + j] = fmaf(__uint_as_float(v[j]), sw1 * s, acc1[c * 16 + j]);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pempty[pb]);
+      }
+      if (!ok) break;
+
+      const int feat = un.mt * 128 + q * 32 + lane;
+      if (GATED) {
+        // h = silu(g) * u, then per-row e4m3 quantisation over this tile's 128 features
+        uint8_t* hq = static_cast<uint8_t*>(args.out);
+#pragma unroll
+        for (int j = 0; j < BN; ++j) {
+          const float gv = acc0[j];
+          acc0[j] = gv / (1.f + expf(-gv)) * acc1[j];
+          if (j < un.nvalid) {
+            const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(acc0[j])));
+            if (lane == 0) amax_s[q * BN + j] = __uint_as_float(m);
+          }
+        }
+        if (!group_sync()) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int j = 0; j < BN; ++j) {
+          if (j < un.nvalid) {
+            const float amax = fmaxf(fmaxf(amax_s[j], amax_s[BN + j]),
+                                     fmaxf(amax_s[2 * BN + j], amax_s[3 * BN + j]));
+            const float sh = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+            const size_t row = static_cast<size_t>(un.row0 + j);
+            float2 pair;
+            pair.x = __fdiv_rn(acc0[j], sh);
+            pair.y = 0.f;
+            const __nv_fp8x2_storage_t b = __nv_cvt_float2_to_fp8x2(pair, __NV_SATFINITE, __NV_E4M3);
+            hq[row * args.ld + feat] = static_cast<uint8_t>(b & 0xFF);
+            if (ptid == 0) args.out_scale[row * args.m_tiles + un.mt] = sh;
+          }
+        }
+      } else {
+        float* out = static_cast<float*>(args.out);
+#pragma unroll
+        for (int j = 0; j < BN; ++j)
+          if (j < un.nvalid) out[static_cast<size_t>(un.row0 + j) * args.ld + feat] = acc0[j];
+      }
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      atomicOr(args.status, MOE_DEVICE_WAIT_TIMEOUT);
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && warp == 0 && lane == 0) {
+    for (uint32_t j = *consumed; j < *issued; ++j)
+      mbar_wait(&full[j % C::kStages], (j / C::kStages) & 1u, nullptr);
+  }
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+template <int BN, bool GATED>
+static cudaError_t launch_one(moe_handle* h, const CUtensorMap& a0, const CUtensorMap& a1,
+                              const CUtensorMap& b, const GemmArgs& args, cudaStream_t s) {
+  using C = Fp8Cfg<BN, GATED>;
+  static bool configured[64] = {};
+  if (h->device < 64 && !configured[h->device]) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_fp8_kernel<BN, GATED>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (e != cudaSuccess) return e;
+    configured[h->device] = true;
+  }
+  grouped_gemm_fp8_kernel<BN, GATED><<<h->num_sms, 192, C::kSmem, s>>>(a0, a1, b, args);
+  h->launches++;
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaStream_t s) {
-  (void)h; (void)gated; (void)p; (void)s;
-  return cudaErrorNotSupported;
+  const Dims& dm = h->dims;
+  if (p.k_blocks > kFp8MaxKBlocks) return cudaErrorInvalidValue;
+  GemmArgs a{};
+  a.offsets = h->ws.offsets;
+  a.unit_base = h->ws.unit_base + (gated ? 0 : (dm.G + 1));
+  a.G = dm.G;
+  a.m_tiles = p.m_tiles;
+  a.k_blocks = p.k_blocks;
+  a.bn = p.bn;
+  a.status = h->ws.status;
+  const int bi = bn_index(p.bn);
+  if (gated) {
+    a.out = h->ws.hbuf;
+    a.ld = dm.f;
+    a.out_scale = h->ws.hs;
+    a.w_scale0 = h->w.gate_s;
+    a.w_scale1 = h->w.up_s;
+    a.act_scale = h->ws.xs;
+    const CUtensorMap& b = h->tm_xp[bi];
+    switch (p.bn) {
+      case 16: return launch_one<16, true>(h, h->tm_gate, h->tm_up, b, a, s);
+      case 32: return launch_one<32, true>(h, h->tm_gate, h->tm_up, b, a, s);
+      case 64: return launch_one<64, true>(h, h->tm_gate, h->tm_up, b, a, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  a.out = h->ws.out;
+  a.ld = dm.d;
+  a.w_scale0 = h->w.down_s;
+  a.w_scale1 = h->w.down_s;
+  a.act_scale = h->ws.hs;
+  const CUtensorMap& b = h->tm_h[bi];
+  switch (p.bn) {
+    case 16: return launch_one<16, false>(h, h->tm_down, h->tm_down, b, a, s);
+    case 32: return launch_one<32, false>(h, h->tm_down, h->tm_down, b, a, s);
+    case 64: return launch_one<64, false>(h, h->tm_down, h->tm_down, b, a, s);
+    case 128: return launch_one<128, false>(h, h->tm_down, h->tm_down, b, a, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace smoe

@@ -105,6 +105,8 @@ cudaError_t launch_route_scan(moe_handle* h, int T, const GemmPlan& p1, const Ge
                               cudaStream_t s);
 cudaError_t launch_dispatch(moe_handle* h, const void* x, int T, cudaStream_t s);
 cudaError_t launch_combine(moe_handle* h, void* y, int T, cudaStream_t s);
+cudaError_t launch_act_quant(const void* x, int64_t rows, int d, uint8_t* q, float* s,
+                             cudaStream_t st);
 // gemm_bf16.cu / gemm_fp8.cu
 cudaError_t launch_gemm_bf16(moe_handle* h, bool gated, const GemmPlan& p, cudaStream_t s);
 cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaStream_t s);
