@@ -47,8 +47,8 @@ METRIC = "K2 MoE layer tokens/s; % of HBM (decode) / tensor-peak (prefill) roofl
 UNIT = "tokens/s"
 PHASES = ("router_logits", "router_topk", "route_scan", "dispatch", "gemm_gate_up",
           "gemm_down", "combine")
-KERNEL_SOURCES = {"gemm_gate_up": ["gemm_bf16.cu", "gemm_fp8.cu", "gemm_common.cuh", "sm100.cuh"],
-                  "gemm_down": ["gemm_bf16.cu", "gemm_fp8.cu", "gemm_common.cuh", "sm100.cuh"]}
+KERNEL_SOURCES = {"gemm_gate_up": ["gemm_bf16.cu", "gemm_promoted.cu", "gemm_common.cuh", "sm100.cuh"],
+                  "gemm_down": ["gemm_bf16.cu", "gemm_promoted.cu", "gemm_common.cuh", "sm100.cuh"]}
 
 
 # ----------------------------------------------------------------- workloads

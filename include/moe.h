@@ -123,6 +123,7 @@ typedef struct {
                                      selecting (weights still from the unbiased scores);
                                      ids must be distinct per token and < E, else the
                                      status word gets MOE_DEVICE_BAD_EXPERT_ID */
+  float* router_logits_out;       /* optional device [T, E]: the router logits x . W_g^T */
   uint32_t flags;                 /* MOE_FLAG_* */
 } moe_forward_opts_t;
 

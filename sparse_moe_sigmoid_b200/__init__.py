@@ -62,7 +62,8 @@ class moe_weights_t(ctypes.Structure):
 
 class moe_forward_opts_t(ctypes.Structure):
     _fields_ = [("topk_ids_out", ctypes.c_void_p), ("topk_weights_out", ctypes.c_void_p),
-                ("forced_topk_ids", ctypes.c_void_p), ("flags", ctypes.c_uint32)]
+                ("forced_topk_ids", ctypes.c_void_p), ("router_logits_out", ctypes.c_void_p),
+                ("flags", ctypes.c_uint32)]
 
 
 _H = ctypes.c_void_p
@@ -164,19 +165,21 @@ def moe_load_weights(h, router_weight, e_score_correction_bias, gate_proj, up_pr
     _check(_lib.moe_load_weights(h, ctypes.byref(w), _stream(stream)), "moe_load_weights", h)
 
 
-def _opts(topk_ids_out, topk_weights_out, forced_topk_ids, flags):
-    if topk_ids_out is None and topk_weights_out is None and forced_topk_ids is None and not flags:
+def _opts(topk_ids_out, topk_weights_out, forced_topk_ids, router_logits_out, flags):
+    if (topk_ids_out is None and topk_weights_out is None and forced_topk_ids is None
+            and router_logits_out is None and not flags):
         return None
     return ctypes.byref(moe_forward_opts_t(_ptr(topk_ids_out), _ptr(topk_weights_out),
-                                           _ptr(forced_topk_ids), flags))
+                                           _ptr(forced_topk_ids), _ptr(router_logits_out), flags))
 
 
 def moe_forward(h, x, y, T: Optional[int] = None, topk_ids_out=None, topk_weights_out=None,
-                forced_topk_ids=None, flags: int = 0, stream=None):
+                forced_topk_ids=None, router_logits_out=None, flags: int = 0, stream=None):
     """y = MoE(x); x and y are BF16 [T, hidden] device tensors."""
     T = x.shape[0] if T is None else T
     st = _lib.moe_forward(h, _ptr(x), T, _ptr(y),
-                          _opts(topk_ids_out, topk_weights_out, forced_topk_ids, flags),
+                          _opts(topk_ids_out, topk_weights_out, forced_topk_ids,
+                                router_logits_out, flags),
                           _stream(stream))
     _check(st, "moe_forward", h)
 
@@ -185,7 +188,7 @@ def moe_forward_host(h, x_host, y_host, T: Optional[int] = None, flags: int = 0,
     """The same from host (CPU, ideally pinned) BF16 tensors; synchronises."""
     T = x_host.shape[0] if T is None else T
     st = _lib.moe_forward_host(h, _ptr(x_host), T, _ptr(y_host),
-                               _opts(None, None, None, flags), _stream(stream))
+                               _opts(None, None, None, None, flags), _stream(stream))
     _check(st, "moe_forward_host", h)
 
 

@@ -158,7 +158,7 @@ void free_all(moe_handle* h) {
   auto f = [](void* p) {
     if (p) cudaFree(p);
   };
-  f(h->w.router); f(h->w.bias); f(h->w.gate); f(h->w.up); f(h->w.down);
+  f(h->w.router); f(h->w.router_cat); f(h->w.bias); f(h->w.gate); f(h->w.up); f(h->w.down);
   f(h->w.gate_s); f(h->w.up_s); f(h->w.down_s);
   f(h->ws.logits_part); f(h->ws.ids); f(h->ws.wts); f(h->ws.counts); f(h->ws.word_prefix);
   f(h->ws.offsets); f(h->ws.unit_base); f(h->ws.pair_row); f(h->ws.row_token); f(h->ws.xp);
@@ -245,6 +245,7 @@ moe_status_t moe_create(const moe_config_t* cfg, int device, moe_handle_t** out)
     if (e != cudaSuccess) rc = cuda_fail(h, e, what);
   };
   A(&h->w.router, E * d * 4, "router weight");
+  A(&h->w.router_cat, E * 3 * d * 2, "router weight split");
   A(&h->w.bias, E * 4, "bias");
   A(&h->w.gate, G * f * d * wb, "gate_proj");
   A(&h->w.up, G * f * d * wb, "up_proj");
@@ -308,6 +309,13 @@ moe_status_t moe_create(const moe_config_t* cfg, int device, moe_handle_t** out)
     uint32_t box[3] = {kbox, 128, 1};
     ok = ok && smoe::make_tmap(&h->tm_down, dt, 3, h->w.down, dims, str, box, &why);
   }
+  {
+    uint64_t dims[3] = {3 * d, E, 1};
+    uint64_t str[2] = {3 * d * 2, E * 3 * d * 2};
+    uint32_t box[3] = {64, 128, 1};
+    ok = ok && smoe::make_tmap(&h->tm_router, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, h->w.router_cat,
+                               dims, str, box, &why);
+  }
   for (int i = 0; i < 5 && ok; ++i) {
     const uint32_t bn = 16u << i;
     uint64_t dx[2] = {d, Rm};
@@ -352,6 +360,7 @@ moe_status_t moe_load_weights(moe_handle_t* h, const moe_weights_t* w, void* str
 
   CUDA_TRY(h, cudaMemcpyAsync(h->w.router, w->router_weight, E * d * 4, K, s), "router copy");
   CUDA_TRY(h, cudaMemcpyAsync(h->w.bias, w->e_score_correction_bias, E * 4, K, s), "bias copy");
+  CUDA_TRY(h, smoe::launch_router_split(h, s), "router split launch");
   CUDA_TRY(h, cudaMemcpyAsync(h->w.gate, w->gate_proj, E * f * d * wb, K, s), "gate copy");
   CUDA_TRY(h, cudaMemcpyAsync(h->w.up, w->up_proj, E * f * d * wb, K, s), "up copy");
   CUDA_TRY(h, cudaMemcpyAsync(h->w.down, w->down_proj, E * d * f * wb, K, s), "down copy");
@@ -436,10 +445,17 @@ moe_status_t moe_forward(moe_handle_t* h, const void* x, int64_t T, void* y,
 
   mark(0);
   CUDA_TRY(h, cudaMemsetAsync(h->ws.counts, 0, h->ws.zero_bytes, s), "clear counts");
-  CUDA_TRY(h, smoe::launch_router_logits(h, x, Ti, splits, s), "router logits launch");
+  const bool tensor_router = T >= smoe::kTensorRouterMinT;
+  if (tensor_router) {
+    CUDA_TRY(h, smoe::launch_router_gemm(h, x, Ti, s), "router GEMM launch");
+  } else {
+    CUDA_TRY(h, smoe::launch_router_logits(h, x, Ti, splits, s), "router logits launch");
+  }
   mark(1);
-  CUDA_TRY(h, smoe::launch_router_topk(h, Ti, splits, forced, s, opts ? opts->topk_ids_out : nullptr,
-                                       opts ? opts->topk_weights_out : nullptr),
+  CUDA_TRY(h, smoe::launch_router_topk(h, Ti, tensor_router ? 1 : splits, forced, s,
+                                       opts ? opts->topk_ids_out : nullptr,
+                                       opts ? opts->topk_weights_out : nullptr,
+                                       opts ? opts->router_logits_out : nullptr),
            "router top-k launch");
   mark(2);
   CUDA_TRY(h, smoe::launch_route_scan(h, Ti, p1, p2, s), "route scan launch");

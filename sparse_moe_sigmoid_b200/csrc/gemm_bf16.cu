@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total_units = __ldg(args.unit_base + args.G);
+  const int total_units = total_units_of(args, BN);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(192, 1)
           mbar_arrive_expect_tx(&full[s], C::kStage);
           tma_load_3d(st, &tmA0, &full[s], kb * 64, un.mt * 128, un.g);
           if (GATED) tma_load_3d(st + C::kA, &tmA1, &full[s], kb * 64, un.mt * 128, un.g);
-          tma_load_2d(st + C::kA * C::kNumA, &tmB, &full[s], kb * 64, un.row0);
+          tma_load_2d(st + C::kA * C::kNumA, &tmB, &full[s], (kb * 64) % args.b_k, un.row0);
           *issued = it + 1;
         }
       }
@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(192, 1)
               const float uv = __uint_as_float(v[j]);
               const float hv = gv / (1.f + expf(-gv)) * uv;
               static_cast<__nv_bfloat16*>(args.out)[row * args.ld + feat] = __float2bfloat16_rn(hv);
-            } else {
+            } else if (feat < args.m_valid) {
               static_cast<float*>(args.out)[row * args.ld + feat] = __uint_as_float(g[j]);
             }
           }
@@ -266,6 +266,8 @@ cudaError_t launch_gemm_bf16(moe_handle* h, bool gated, const GemmPlan& p, cudaS
   a.k_blocks = p.k_blocks;
   a.bn = p.bn;
   a.status = h->ws.status;
+  a.b_k = gated ? dm.d : dm.f;
+  a.m_valid = p.m_tiles * 128;
   const int bi = bn_index(p.bn);
   if (gated) {
     a.out = h->ws.hbuf;

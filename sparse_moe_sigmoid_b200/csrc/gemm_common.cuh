@@ -36,9 +36,27 @@ struct GemmArgs {
   const float* w_scale1;     // FP8 gate/up: of A1
   const float* act_scale;    // FP8: activation scales [R][k_blocks]
   uint32_t* status;
+  int single_rows;           // unit_base == nullptr: one group of this many rows at row 0
+  int b_k;                   // K extent of B; the K index into B is (k mod b_k)
+  int m_valid;               // only output features < m_valid are stored
+  int kpp;                   // promoted BF16 GEMM: stages accumulated in TMEM per promotion
 };
 
+__device__ __forceinline__ int total_units_of(const GemmArgs& a, int BN) {
+  return a.unit_base ? __ldg(a.unit_base + a.G) : a.m_tiles * ((a.single_rows + BN - 1) / BN);
+}
+
 __device__ __forceinline__ Unit decode_unit(int u, const GemmArgs& a, int BN) {
+  Unit un;
+  if (a.unit_base == nullptr) {
+    const int nt = (a.single_rows + BN - 1) / BN;
+    un.g = 0;
+    un.mt = u / nt;
+    const int ti = u - un.mt * nt;
+    un.row0 = ti * BN;
+    un.nvalid = min(BN, a.single_rows - ti * BN);
+    return un;
+  }
   // last group whose first unit is <= u (empty groups own no units)
   int lo = 0, hi = a.G;
   while (hi - lo > 1) {
@@ -46,7 +64,6 @@ __device__ __forceinline__ Unit decode_unit(int u, const GemmArgs& a, int BN) {
     if (__ldg(a.unit_base + mid) <= u) lo = mid;
     else hi = mid;
   }
-  Unit un;
   un.g = lo;
   const int r0 = __ldg(a.offsets + lo);
   const int cnt = __ldg(a.offsets + lo + 1) - r0;

@@ -23,6 +23,14 @@
 // conversion), written with its scale for the down GEMM.
 // Down epilogue: the promoted fp32 row outputs.
 //
+// The same kernel with BF16 operands and no scales computes the router
+// logits on the tensor cores (launch_router_gemm below): there the point of
+// promoting every 128 K is precision, not scaling. The tensor core adds each
+// MMA's products into its fp32 accumulator with a rounding that, over
+// K = 3 x 7168, drifts by more than the 1e-5 band in which the top-k choice
+// may legitimately differ; partial sums over 128 K stay small (so their
+// rounding is tiny) and are added in fp32 registers with round-to-nearest.
+//
 // Roles and the bounded-wait / wind-down rules are those of the BF16 kernel
 // (gemm_bf16.cu): warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
 // warps 2..5 promotion + epilogue.
@@ -38,14 +46,17 @@ using namespace sm100;
 
 constexpr int kFp8MaxKBlocks = 64;  // hidden_size and moe_intermediate_size <= 8192
 
-template <int BN, bool GATED>
-struct Fp8Cfg {
-  static constexpr int kA = 128 * 128;  // 128 rows x 128 e4m3
+// FP8: e4m3 operands, 128 K per stage, block scales applied at promotion.
+// Otherwise BF16 operands, 64 K per stage, no scales.
+template <int BN, bool GATED, bool FP8>
+struct PromCfg {
+  static constexpr int kA = 128 * 128;  // 128 rows x 128 bytes of K
   static constexpr int kB = BN * 128;
+  static constexpr int kKPerStage = FP8 ? 128 : 64;
   static constexpr int kNumA = GATED ? 2 : 1;
   static constexpr int kStage = kA * kNumA + kB;
-  static constexpr int kScaleBytes = (kFp8MaxKBlocks * BN + 2 * kFp8MaxKBlocks) * 4;
-  static constexpr int kAmaxBytes = 4 * BN * 4;
+  static constexpr int kScaleBytes = FP8 ? (kFp8MaxKBlocks * BN + 2 * kFp8MaxKBlocks) * 4 : 0;
+  static constexpr int kAmaxBytes = GATED ? 4 * BN * 4 : 0;
   static constexpr int kStages0 = (227 * 1024 - 2048 - kScaleBytes - kAmaxBytes) / kStage;
   static constexpr int kStages = kStages0 > 10 ? 10 : kStages0;
   static constexpr int kPCols = GATED ? 2 * BN : BN;  // one partial buffer
@@ -55,19 +66,20 @@ struct Fp8Cfg {
   static_assert(kStages >= 2, "need at least two stages");
 };
 
-template <int BN, bool GATED>
+template <int BN, bool GATED, bool FP8>
 __global__ void __launch_bounds__(192, 1)
-    grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA0,
-                            const __grid_constant__ CUtensorMap tmA1,
-                            const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
-  using C = Fp8Cfg<BN, GATED>;
+    grouped_gemm_promoted_kernel(const __grid_constant__ CUtensorMap tmA0,
+                                 const __grid_constant__ CUtensorMap tmA1,
+                                 const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+  using C = PromCfg<BN, GATED, FP8>;
+  static_assert(FP8 || !GATED, "the BF16 promoted GEMM is plain");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  float* sa_s = reinterpret_cast<float*>(smem + C::kStages * C::kStage);  // [KB][BN]
-  float* sw_s = sa_s + kFp8MaxKBlocks * BN;                                // [2][KB]
-  float* amax_s = sw_s + 2 * kFp8MaxKBlocks;                               // [4][BN]
-  uint64_t* full = reinterpret_cast<uint64_t*>(amax_s + 4 * BN);
+  float* sa_s = reinterpret_cast<float*>(smem + C::kStages * C::kStage);  // [KB][BN] (FP8)
+  float* sw_s = sa_s + (FP8 ? kFp8MaxKBlocks * BN : 0);                    // [2][KB] (FP8)
+  float* amax_s = sw_s + (FP8 ? 2 * kFp8MaxKBlocks : 0);                   // [4][BN] (gated)
+  uint64_t* full = reinterpret_cast<uint64_t*>(amax_s + (GATED ? 4 * BN : 0));
   uint64_t* empty = full + C::kStages;
   uint64_t* pfull = empty + C::kStages;
   uint64_t* pempty = pfull + 2;
@@ -81,6 +93,7 @@ __global__ void __launch_bounds__(192, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int KB = args.k_blocks;
+  const int KPP = FP8 ? 1 : args.kpp;  // stages accumulated per promotion
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -112,7 +125,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total_units = __ldg(args.unit_base + args.G);
+  const int total_units = total_units_of(args, BN);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -129,9 +142,10 @@ __global__ void __launch_bounds__(192, 1)
           }
           uint8_t* st = smem + s * C::kStage;
           mbar_arrive_expect_tx(&full[s], C::kStage);
-          tma_load_3d(st, &tmA0, &full[s], kb * 128, un.mt * 128, un.g);
-          if (GATED) tma_load_3d(st + C::kA, &tmA1, &full[s], kb * 128, un.mt * 128, un.g);
-          tma_load_2d(st + C::kA * C::kNumA, &tmB, &full[s], kb * 128, un.row0);
+          const int kc = kb * C::kKPerStage;
+          tma_load_3d(st, &tmA0, &full[s], kc, un.mt * 128, un.g);
+          if (GATED) tma_load_3d(st + C::kA, &tmA1, &full[s], kc, un.mt * 128, un.g);
+          tma_load_2d(st + C::kA * C::kNumA, &tmB, &full[s], kc % args.b_k, un.row0);
           *issued = it + 1;
         }
       }
@@ -142,17 +156,19 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      uint32_t it = 0;  // k-blocks issued so far (also the partial-buffer sequence)
+      uint32_t it = 0;   // stages consumed so far
+      uint32_t pit = 0;  // promotions handed over so far (the partial-buffer sequence)
       bool ok = true;
       for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
         const Unit un = decode_unit(u, args, BN);
         const uint32_t n = static_cast<uint32_t>(((un.nvalid + 15) / 16) * 16);
-        const uint32_t idesc = make_idesc(0u, n);
+        const uint32_t idesc = make_idesc(FP8 ? 0u : 1u, n);
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % C::kStages;
           const uint32_t ph = (it / C::kStages) & 1u;
-          const int pb = it & 1;
-          if (!mbar_wait(&pempty[pb], ((it >> 1) & 1u) ^ 1u, abort_flag) ||
+          const int pb = pit & 1;
+          const int sub = kb % KPP;
+          if ((sub == 0 && !mbar_wait(&pempty[pb], ((pit >> 1) & 1u) ^ 1u, abort_flag)) ||
               !mbar_wait(&full[s], ph, abort_flag)) {
             ok = false;
             break;
@@ -165,12 +181,19 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t d0 = tmem_base + pb * C::kPCols;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const uint32_t accum = k ? 1u : 0u;  // each block's partial starts fresh
-            mma_fp8(d0, ad0 + 2 * k, bd + 2 * k, idesc, accum);
-            if (GATED) mma_fp8(d0 + BN, ad1 + 2 * k, bd + 2 * k, idesc, accum);
+            const uint32_t accum = (k | sub) ? 1u : 0u;  // each promotion's partial starts fresh
+            if (FP8) {
+              mma_fp8(d0, ad0 + 2 * k, bd + 2 * k, idesc, accum);
+              if (GATED) mma_fp8(d0 + BN, ad1 + 2 * k, bd + 2 * k, idesc, accum);
+            } else {
+              mma_bf16(d0, ad0 + 2 * k, bd + 2 * k, idesc, accum);
+            }
           }
           mma_commit(&empty[s]);
-          mma_commit(&pfull[pb]);
+          if (sub == KPP - 1 || kb == KB - 1) {
+            mma_commit(&pfull[pb]);
+            ++pit;
+          }
           *consumed = it + 1;
         }
       }
@@ -184,7 +207,7 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     const int q = warp & 3;           // TMEM lane quarter
     const int ptid = threadIdx.x - 64;  // 0..127 among the promotion warps
-    uint32_t it = 0, gph = 0;
+    uint32_t pit = 0, gph = 0;
     bool ok = true;
     auto group_sync = [&]() {
       mbar_arrive(grp);
@@ -192,25 +215,28 @@ __global__ void __launch_bounds__(192, 1)
       gph ^= 1u;
       return r;
     };
+    const int NP = (KB + KPP - 1) / KPP;  // promotions per tile
     for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
       const Unit un = decode_unit(u, args, BN);
-      // this tile's scales: activations [KB][BN] and the weight block scales
-      if (!group_sync()) {  // the previous tile's readers are done
-        ok = false;
-        break;
-      }
-      for (int i = ptid; i < KB * BN; i += 128) {
-        const int kb = i / BN, j = i - kb * BN;
-        sa_s[i] = j < un.nvalid ? __ldg(args.act_scale + (size_t)(un.row0 + j) * KB + kb) : 0.f;
-      }
-      const size_t wrow = ((size_t)un.g * args.m_tiles + un.mt) * KB;
-      for (int i = ptid; i < KB; i += 128) {
-        sw_s[i] = __ldg(args.w_scale0 + wrow + i);
-        if (GATED) sw_s[kFp8MaxKBlocks + i] = __ldg(args.w_scale1 + wrow + i);
-      }
-      if (!group_sync()) {
-        ok = false;
-        break;
+      if (FP8) {
+        // this tile's scales: activations [KB][BN] and the weight block scales
+        if (!group_sync()) {  // the previous tile's readers are done
+          ok = false;
+          break;
+        }
+        for (int i = ptid; i < KB * BN; i += 128) {
+          const int kb = i / BN, j = i - kb * BN;
+          sa_s[i] = j < un.nvalid ? __ldg(args.act_scale + (size_t)(un.row0 + j) * KB + kb) : 0.f;
+        }
+        const size_t wrow = ((size_t)un.g * args.m_tiles + un.mt) * KB;
+        for (int i = ptid; i < KB; i += 128) {
+          sw_s[i] = __ldg(args.w_scale0 + wrow + i);
+          if (GATED) sw_s[kFp8MaxKBlocks + i] = __ldg(args.w_scale1 + wrow + i);
+        }
+        if (!group_sync()) {
+          ok = false;
+          break;
+        }
       }
 
       float acc0[BN], acc1[GATED ? BN : 1];
@@ -220,16 +246,16 @@ __global__ void __launch_bounds__(192, 1)
         if (GATED) acc1[j] = 0.f;
       }
       const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-      for (int kb = 0; kb < KB; ++kb, ++it) {
-        const int pb = it & 1;
-        if (!mbar_wait(&pfull[pb], (it >> 1) & 1u, abort_flag)) {
+      for (int pg = 0; pg < NP; ++pg, ++pit) {
+        const int pb = pit & 1;
+        if (!mbar_wait(&pfull[pb], (pit >> 1) & 1u, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const float sw0 = sw_s[kb];
-        const float sw1 = GATED ? sw_s[kFp8MaxKBlocks + kb] : 0.f;
-        const float* sa = sa_s + kb * BN;
+        const float sw0 = FP8 ? sw_s[pg] : 1.f;
+        const float sw1 = (FP8 && GATED) ? sw_s[kFp8MaxKBlocks + pg] : 0.f;
+        const float* sa = sa_s + pg * BN;
 #pragma unroll
         for (int c = 0; c < BN / 16; ++c) {
           if (c * 16 < un.nvalid) {
@@ -239,9 +265,14 @@ __global__ void __launch_bounds__(192, 1)
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              const float s = sa[c * 16 + j];
-              acc0[c * 16 + j] = fmaf(__uint_as_float(g[j]), sw0 * s, acc0[c * 16 + j]);
-              if (GATED) acc1[c * 16 + j] = fmaf(__uint_as_float(v[j]), sw1 * s, acc1[c * 16 + j]);
+              if (FP8) {
+                const float s = sa[c * 16 + j];
+                acc0[c * 16 + j] = fmaf(__uint_as_float(g[j]), sw0 * s, acc0[c * 16 + j]);
+                if (GATED)
+                  acc1[c * 16 + j] = fmaf(__uint_as_float(v[j]), sw1 * s, acc1[c * 16 + j]);
+              } else {
+                acc0[c * 16 + j] += __uint_as_float(g[j]);
+              }
             }
           }
         }
@@ -285,9 +316,11 @@ __global__ void __launch_bounds__(192, 1)
         }
       } else {
         float* out = static_cast<float*>(args.out);
+        if (feat < args.m_valid) {
 #pragma unroll
-        for (int j = 0; j < BN; ++j)
-          if (j < un.nvalid) out[static_cast<size_t>(un.row0 + j) * args.ld + feat] = acc0[j];
+          for (int j = 0; j < BN; ++j)
+            if (j < un.nvalid) out[static_cast<size_t>(un.row0 + j) * args.ld + feat] = acc0[j];
+        }
       }
     }
     if (!ok && lane == 0) {
@@ -308,18 +341,18 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
-template <int BN, bool GATED>
+template <int BN, bool GATED, bool FP8 = true>
 static cudaError_t launch_one(moe_handle* h, const CUtensorMap& a0, const CUtensorMap& a1,
                               const CUtensorMap& b, const GemmArgs& args, cudaStream_t s) {
-  using C = Fp8Cfg<BN, GATED>;
+  using C = PromCfg<BN, GATED, FP8>;
   static bool configured[64] = {};
   if (h->device < 64 && !configured[h->device]) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_fp8_kernel<BN, GATED>,
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_promoted_kernel<BN, GATED, FP8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
     configured[h->device] = true;
   }
-  grouped_gemm_fp8_kernel<BN, GATED><<<h->num_sms, 192, C::kSmem, s>>>(a0, a1, b, args);
+  grouped_gemm_promoted_kernel<BN, GATED, FP8><<<h->num_sms, 192, C::kSmem, s>>>(a0, a1, b, args);
   h->launches++;
   return cudaGetLastError();
 }
@@ -335,6 +368,8 @@ cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaSt
   a.k_blocks = p.k_blocks;
   a.bn = p.bn;
   a.status = h->ws.status;
+  a.b_k = gated ? dm.d : dm.f;
+  a.m_valid = p.m_tiles * 128;
   const int bi = bn_index(p.bn);
   if (gated) {
     a.out = h->ws.hbuf;
@@ -364,6 +399,42 @@ cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaSt
     case 128: return launch_one<128, false>(h, h->tm_down, h->tm_down, b, a, s);
     default: return cudaErrorInvalidValue;
   }
+}
+
+// Router logits on the tensor cores: logits[t, e] = x_t . W_g[e] with the fp32
+// router weight held as three BF16 parts W = hi + mid + lo (exact: 3 x 8
+// significand bits cover fp32's 24), concatenated along K. x (BF16) times
+// each part is an exact product; partial sums over 128 K are promoted into
+// fp32 registers (see the file comment). One group of T rows; B's K index
+// wraps onto x's d columns.
+cudaError_t launch_router_gemm(moe_handle* h, const void* x, int T, cudaStream_t s) {
+  const Dims& dm = h->dims;
+  constexpr int BN = 128;
+  CUtensorMap tmx;
+  {
+    uint64_t dims[2] = {static_cast<uint64_t>(dm.d), static_cast<uint64_t>(T)};
+    uint64_t str[1] = {static_cast<uint64_t>(dm.d) * 2};
+    uint32_t box[2] = {64, BN};
+    std::string err;
+    if (!make_tmap(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, str, box,
+                   &err))
+      return cudaErrorInvalidValue;
+  }
+  GemmArgs a{};
+  a.offsets = nullptr;
+  a.unit_base = nullptr;
+  a.G = 1;
+  a.single_rows = T;
+  a.m_tiles = (dm.E + 127) / 128;
+  a.k_blocks = 3 * dm.d / 64;
+  a.kpp = 2;
+  a.bn = BN;
+  a.b_k = dm.d;
+  a.m_valid = dm.E;
+  a.out = h->ws.logits_part;
+  a.ld = dm.E;
+  a.status = h->ws.status;
+  return launch_one<BN, false, false>(h, h->tm_router, h->tm_router, tmx, a, s);
 }
 
 }  // namespace smoe

@@ -17,6 +17,7 @@ constexpr int kMaxTopK = 32;
 constexpr int kMaxExperts = 512;
 constexpr int kRouterTile = 64;   // router tile: 64 tokens x 64 experts
 constexpr int kRouterKTile = 32;
+constexpr int kRouterMaxSplits = 16;
 
 // Sizes derived from the config, fixed per handle.
 struct Dims {
@@ -56,6 +57,7 @@ struct Workspace {
 
 struct Weights {
   float* router = nullptr;  // [E][d]
+  void* router_cat = nullptr;  // [E][3d] BF16: W_g = hi + mid + lo
   float* bias = nullptr;    // [E]
   void* gate = nullptr;     // [G][f][d]
   void* up = nullptr;       // [G][f][d]
@@ -77,7 +79,7 @@ struct moe_handle {
   smoe::Workspace ws;
   // TMA descriptors: weights (one per projection) and the two activation
   // matrices, the latter once per supported row-tile height (16 << i)
-  CUtensorMap tm_gate, tm_up, tm_down;
+  CUtensorMap tm_gate, tm_up, tm_down, tm_router;
   CUtensorMap tm_xp[5], tm_h[5];
   int router_max_splits = 1;
   int64_t launches = 0;
@@ -93,7 +95,12 @@ namespace smoe {
 int router_splits(const Dims& dm, int64_t T, int num_sms);
 cudaError_t launch_router_logits(moe_handle* h, const void* x, int T, int splits, cudaStream_t s);
 cudaError_t launch_router_topk(moe_handle* h, int T, int splits, const int32_t* forced,
-                               cudaStream_t s, int32_t* ids_out, float* wts_out);
+                               cudaStream_t s, int32_t* ids_out, float* wts_out,
+                               float* logits_out);
+cudaError_t launch_router_split(moe_handle* h, cudaStream_t s);
+// gemm_promoted.cu: the router's logits on the tensor cores (T >= kTensorRouterMinT)
+cudaError_t launch_router_gemm(moe_handle* h, const void* x, int T, cudaStream_t s);
+constexpr int kTensorRouterMinT = 512;
 cudaError_t launch_router_raw(const void* x, const float* router_weight, const float* bias, int T,
                               int d, int E, int k, float scale, int norm, int splits, float* part,
                               int32_t* counts, uint32_t* bitmap, int W, uint32_t* status,
@@ -107,7 +114,7 @@ cudaError_t launch_dispatch(moe_handle* h, const void* x, int T, cudaStream_t s)
 cudaError_t launch_combine(moe_handle* h, void* y, int T, cudaStream_t s);
 cudaError_t launch_act_quant(const void* x, int64_t rows, int d, uint8_t* q, float* s,
                              cudaStream_t st);
-// gemm_bf16.cu / gemm_fp8.cu
+// gemm_bf16.cu / gemm_promoted.cu
 cudaError_t launch_gemm_bf16(moe_handle* h, bool gated, const GemmPlan& p, cudaStream_t s);
 cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaStream_t s);
 int bn_index(int bn);

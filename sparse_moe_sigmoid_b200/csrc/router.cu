@@ -30,7 +30,9 @@ int router_splits(const Dims& dm, int64_t T, int num_sms) {
   const int64_t tiles = ((dm.E + kRouterTile - 1) / kRouterTile) *
                         ((T + kRouterTile - 1) / kRouterTile);
   int64_t want = (2 * num_sms + tiles - 1) / tiles;
-  int64_t max_splits = dm.d / kRouterKTile;
+  // the top-k kernel adds the slices serially per lane: keep them few
+  int64_t max_splits = dm.d / kRouterKTile < kRouterMaxSplits ? dm.d / kRouterKTile
+                                                               : kRouterMaxSplits;
   if (want < 1) want = 1;
   if (want > max_splits) want = max_splits;
   // each slice is a multiple of the 32-wide K tile
@@ -133,7 +135,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     int k, float scale, int norm, const int32_t* __restrict__ forced, int32_t* __restrict__ ids,
     float* __restrict__ wts, int32_t* __restrict__ counts, uint32_t* __restrict__ bitmap,
     int W, uint32_t* __restrict__ status, int32_t* __restrict__ ids_out,
-    float* __restrict__ wts_out) {
+    float* __restrict__ wts_out, float* __restrict__ logits_out) {
   const int lane = threadIdx.x & 31;
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= T) return;
@@ -146,6 +148,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     if (e < E) {
       float l = 0.f;
       for (int s = 0; s < splits; ++s) l += part[((size_t)s * T + t) * E + e];
+      if (logits_out) logits_out[(size_t)t * E + e] = l;
       const float p = 1.f / (1.f + expf(-l));
       sc[i] = p;
       key[i] = p + bias[e];
@@ -257,14 +260,15 @@ cudaError_t launch_router_logits(moe_handle* h, const void* x, int T, int splits
 }
 
 cudaError_t launch_router_topk(moe_handle* h, int T, int splits, const int32_t* forced,
-                               cudaStream_t s, int32_t* ids_out, float* wts_out) {
+                               cudaStream_t s, int32_t* ids_out, float* wts_out,
+                               float* logits_out) {
   const Dims& dm = h->dims;
   const int W = static_cast<int>((dm.Tmax + 31) / 32);
   const int blocks = (T * 32 + 255) / 256;
   router_topk_kernel<<<blocks, 256, 0, s>>>(
       h->ws.logits_part, splits, h->w.bias, T, dm.E, dm.k, h->cfg.routed_scaling_factor,
       h->cfg.norm_topk_prob, forced, h->ws.ids, h->ws.wts, h->ws.counts, h->ws.bitmap, W,
-      h->ws.status, ids_out, wts_out);
+      h->ws.status, ids_out, wts_out, logits_out);
   h->launches++;
   return cudaGetLastError();
 }
@@ -285,7 +289,37 @@ cudaError_t launch_router_raw(const void* x, const float* router_weight, const f
   if (e != cudaSuccess) return e;
   const int blocks = (T * 32 + 255) / 256;
   router_topk_kernel<<<blocks, 256, 0, s>>>(part, splits, bias, T, E, k, scale, norm, nullptr, ids,
-                                            wts, counts, bitmap, W, status, nullptr, nullptr);
+                                            wts, counts, bitmap, W, status, nullptr, nullptr,
+                                            nullptr);
+  return cudaGetLastError();
+}
+
+// W_g (fp32 [E][d]) -> cat (BF16 [E][3d]) = [hi | mid | lo] with
+// hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid); the differences
+// are exact in fp32 and hi + mid + lo = w.
+__global__ void router_split_kernel(const float* __restrict__ W, __nv_bfloat16* __restrict__ cat,
+                                    int E, int d) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)E * d) return;
+  const int64_t e = i / d, c = i - e * d;
+  const float w = W[i];
+  const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+  const float r1 = w - __bfloat162float(hi);
+  const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(mid);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
+  __nv_bfloat16* row = cat + e * 3 * (int64_t)d;
+  row[c] = hi;
+  row[d + c] = mid;
+  row[2 * d + c] = lo;
+}
+
+cudaError_t launch_router_split(moe_handle* h, cudaStream_t s) {
+  const Dims& dm = h->dims;
+  const int64_t n = (int64_t)dm.E * dm.d;
+  router_split_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
+      h->w.router, static_cast<__nv_bfloat16*>(h->w.router_cat), dm.E, dm.d);
+  h->launches++;
   return cudaGetLastError();
 }
 
