@@ -19,16 +19,7 @@ using smoe::GemmPlan;
 
 namespace smoe {
 
-int bn_index(int bn) {
-  switch (bn) {
-    case 16: return 0;
-    case 32: return 1;
-    case 64: return 2;
-    case 128: return 3;
-    case 256: return 4;
-    default: return -1;
-  }
-}
+int bn_index(int bn) { return (bn >= 16 && bn <= 256 && bn % 16 == 0) ? bn / 16 - 1 : -1; }
 
 using EncodeTiledFn = decltype(&cuTensorMapEncodeTiled);
 
@@ -316,8 +307,8 @@ moe_status_t moe_create(const moe_config_t* cfg, int device, moe_handle_t** out)
     ok = ok && smoe::make_tmap(&h->tm_router, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, h->w.router_cat,
                                dims, str, box, &why);
   }
-  for (int i = 0; i < 5 && ok; ++i) {
-    const uint32_t bn = 16u << i;
+  for (int i = 0; i < 16 && ok; ++i) {
+    const uint32_t bn = 16u * (i + 1);
     uint64_t dx[2] = {d, Rm};
     uint64_t sx[1] = {d * wb};
     uint32_t box[2] = {kbox, bn};

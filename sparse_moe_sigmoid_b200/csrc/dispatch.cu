@@ -34,24 +34,31 @@ static int pick_bn(double want, const int* cands, int n) {
   return cands[n - 1];
 }
 
+// Row-tile height: the smallest supported height >= 1.3 x the mean rows per
+// routed expert, so that nearly every expert's rows fit one tile and each
+// weight slab is read into shared memory once per forward.
 GemmPlan plan_gate_up(const Dims& dm, int64_t T) {
-  static const int bf16_bn[] = {16, 32, 64, 128};
+  static const int bf16_bn[] = {16, 32, 64, 96, 128, 160, 192, 224, 256};
   static const int fp8_bn[] = {16, 32, 64};
-  const double avg = static_cast<double>(T) * dm.k / dm.E;
+  const double want = 1.3 * static_cast<double>(T) * dm.k / dm.E;
   GemmPlan p;
-  p.bn = dm.fp8 ? pick_bn(avg * 1.5, fp8_bn, 3) : pick_bn(avg * 1.5, bf16_bn, 4);
+  p.bn = dm.fp8 ? pick_bn(want, fp8_bn, 3) : pick_bn(want, bf16_bn, 9);
+  p.na = 2;
   p.m_tiles = dm.f / kBlock;
   p.k_blocks = dm.fp8 ? dm.d / 128 : dm.d / 64;
   return p;
 }
 
+// Down projection: with tall row tiles (BF16, BN >= 64) one unit covers 256
+// output features as two 128-row weight tiles sharing the row tile.
 GemmPlan plan_down(const Dims& dm, int64_t T) {
-  static const int bf16_bn[] = {16, 32, 64, 128, 256};
+  static const int bf16_bn[] = {16, 32, 64, 96, 128, 160, 192, 224, 256};
   static const int fp8_bn[] = {16, 32, 64, 128};
-  const double avg = static_cast<double>(T) * dm.k / dm.E;
+  const double want = 1.3 * static_cast<double>(T) * dm.k / dm.E;
   GemmPlan p;
-  p.bn = dm.fp8 ? pick_bn(avg * 1.5, fp8_bn, 4) : pick_bn(avg * 1.5, bf16_bn, 5);
-  p.m_tiles = dm.d / kBlock;
+  p.bn = dm.fp8 ? pick_bn(want, fp8_bn, 4) : pick_bn(want, bf16_bn, 9);
+  p.na = (!dm.fp8 && p.bn >= 64 && dm.d % 256 == 0) ? 2 : 1;
+  p.m_tiles = dm.d / (kBlock * p.na);
   p.k_blocks = dm.fp8 ? dm.f / 128 : dm.f / 64;
   return p;
 }

@@ -40,28 +40,38 @@ namespace smoe {
 
 using namespace sm100;
 
-template <int BN, bool GATED>
+// NA = weight tiles per stage (2: gate and up for SWIGLU, or two 128-row
+// halves of one 256-feature tile for the plain store). The accumulators are
+// double-buffered in TMEM when two sets fit in its 512 columns, else single.
+template <int BN, int NA, bool SWIGLU>
 struct Bf16Cfg {
   static constexpr int kA = 128 * 64 * 2;  // one 128 x 64 BF16 weight tile
   static constexpr int kB = BN * 64 * 2;
-  static constexpr int kNumA = GATED ? 2 : 1;
+  static constexpr int kNumA = NA;
   static constexpr int kStage = kA * kNumA + kB;
   static constexpr int kStages0 = (227 * 1024 - 2048) / kStage;
   static constexpr int kStages = kStages0 > 12 ? 12 : kStages0;
-  static constexpr int kAccCols = GATED ? 2 * BN : BN;
-  static constexpr int kTmemCols = pow2_at_least(2 * kAccCols, 32);
+  static constexpr int kAccCols = NA * BN;
+  static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
+  static constexpr int kTmemCols = pow2_at_least(kAccBufs * kAccCols, 32);
   static constexpr int kSmem = kStages * kStage + 1024 + 256;
   static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(kTmemCols <= 512, "TMEM holds 512 columns");
   static_assert(kStages >= 2, "need at least two stages");
+  static_assert(!SWIGLU || NA == 2, "SwiGLU needs the gate and up tiles");
 };
 
-template <int BN, bool GATED>
+template <int BN, int NA, bool SWIGLU>
 __global__ void __launch_bounds__(192, 1)
     grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA0,
                              const __grid_constant__ CUtensorMap tmA1,
                              const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
-  using C = Bf16Cfg<BN, GATED>;
+  using C = Bf16Cfg<BN, NA, SWIGLU>;
+  // rows of the weight tiles: SwiGLU takes rows [mt*128, +128) of gate (A0)
+  // and up (A1); the plain store with NA = 2 takes rows [mt*256, +256) of
+  // one weight as two halves
+  constexpr int kRowStep = SWIGLU ? 128 : 128 * NA;
+  constexpr int kRow1 = SWIGLU ? 0 : 128;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -83,7 +93,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < C::kAccBufs; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 4);
     }
@@ -96,7 +106,7 @@ __global__ void __launch_bounds__(192, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA0);
-    if (GATED) tma_prefetch_desc(&tmA1);
+    if (NA == 2) tma_prefetch_desc(&tmA1);
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
@@ -124,8 +134,9 @@ __global__ void __launch_bounds__(192, 1)
           }
           uint8_t* st = smem + s * C::kStage;
           mbar_arrive_expect_tx(&full[s], C::kStage);
-          tma_load_3d(st, &tmA0, &full[s], kb * 64, un.mt * 128, un.g);
-          if (GATED) tma_load_3d(st + C::kA, &tmA1, &full[s], kb * 64, un.mt * 128, un.g);
+          tma_load_3d(st, &tmA0, &full[s], kb * 64, un.mt * kRowStep, un.g);
+          if (NA == 2)
+            tma_load_3d(st + C::kA, &tmA1, &full[s], kb * 64, un.mt * kRowStep + kRow1, un.g);
           tma_load_2d(st + C::kA * C::kNumA, &tmB, &full[s], (kb * 64) % args.b_k, un.row0);
           *issued = it + 1;
         }
@@ -142,8 +153,9 @@ __global__ void __launch_bounds__(192, 1)
       int i = 0;
       for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++i) {
         const Unit un = decode_unit(u, args, BN);
-        const int acc = i & 1;
-        if (!mbar_wait(&tempty[acc], ((i >> 1) & 1) ^ 1, abort_flag)) {
+        const int acc = i % C::kAccBufs;
+        const int use = i / C::kAccBufs;
+        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag)) {
           ok = false;
           break;
         }
@@ -168,7 +180,7 @@ __global__ void __launch_bounds__(192, 1)
             const uint32_t accum = (kb | k) ? 1u : 0u;
             // +32 bytes along K inside the swizzled 128-byte row = +2 in addr>>4
             mma_bf16(d0, ad0 + 2 * k, bd + 2 * k, idesc, accum);
-            if (GATED) mma_bf16(d0 + BN, ad1 + 2 * k, bd + 2 * k, idesc, accum);
+            if (NA == 2) mma_bf16(d0 + BN, ad1 + 2 * k, bd + 2 * k, idesc, accum);
           }
           mma_commit(&empty[s]);
           *consumed = it + 1;
@@ -189,8 +201,9 @@ __global__ void __launch_bounds__(192, 1)
     int i = 0;
     for (int u = blockIdx.x; u < total_units; u += gridDim.x, ++i) {
       const Unit un = decode_unit(u, args, BN);
-      const int acc = i & 1;
-      if (!mbar_wait(&tfull[acc], (i >> 1) & 1, abort_flag)) {
+      const int acc = i % C::kAccBufs;
+      const int use = i / C::kAccBufs;
+      if (!mbar_wait(&tfull[acc], use & 1, abort_flag)) {
         if (lane == 0) {
           *abort_flag = 1;
           atomicOr(args.status, MOE_DEVICE_WAIT_TIMEOUT);
@@ -199,24 +212,26 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::kAccCols;
-      const int feat = un.mt * 128 + q * 32 + lane;
+      const int feat = un.mt * kRowStep + q * 32 + lane;
       for (int c0 = 0; c0 < un.nvalid; c0 += 16) {
         uint32_t g[16], v[16];
         tmem_ld16(tb + c0, g);
-        if (GATED) tmem_ld16(tb + BN + c0, v);
+        if (NA == 2) tmem_ld16(tb + BN + c0, v);
         tmem_ld_wait();
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int col = c0 + j;
           if (col < un.nvalid) {
             const size_t row = static_cast<size_t>(un.row0 + col);
-            if (GATED) {
+            if (SWIGLU) {
               const float gv = __uint_as_float(g[j]);
               const float uv = __uint_as_float(v[j]);
               const float hv = gv / (1.f + expf(-gv)) * uv;
               static_cast<__nv_bfloat16*>(args.out)[row * args.ld + feat] = __float2bfloat16_rn(hv);
-            } else if (feat < args.m_valid) {
-              static_cast<float*>(args.out)[row * args.ld + feat] = __uint_as_float(g[j]);
+            } else {
+              float* o = static_cast<float*>(args.out) + row * args.ld;
+              if (feat < args.m_valid) o[feat] = __uint_as_float(g[j]);
+              if (NA == 2 && feat + 128 < args.m_valid) o[feat + 128] = __uint_as_float(v[j]);
             }
           }
         }
@@ -240,18 +255,18 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
-template <int BN, bool GATED>
+template <int BN, int NA, bool SWIGLU>
 static cudaError_t launch_one(moe_handle* h, const CUtensorMap& a0, const CUtensorMap& a1,
                               const CUtensorMap& b, const GemmArgs& args, cudaStream_t s) {
-  using C = Bf16Cfg<BN, GATED>;
+  using C = Bf16Cfg<BN, NA, SWIGLU>;
   static bool configured[64] = {};  // per device ordinal
   if (h->device < 64 && !configured[h->device]) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_bf16_kernel<BN, GATED>,
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_bf16_kernel<BN, NA, SWIGLU>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
     configured[h->device] = true;
   }
-  grouped_gemm_bf16_kernel<BN, GATED><<<h->num_sms, 192, C::kSmem, s>>>(a0, a1, b, args);
+  grouped_gemm_bf16_kernel<BN, NA, SWIGLU><<<h->num_sms, 192, C::kSmem, s>>>(a0, a1, b, args);
   h->launches++;
   return cudaGetLastError();
 }
@@ -267,29 +282,47 @@ cudaError_t launch_gemm_bf16(moe_handle* h, bool gated, const GemmPlan& p, cudaS
   a.bn = p.bn;
   a.status = h->ws.status;
   a.b_k = gated ? dm.d : dm.f;
-  a.m_valid = p.m_tiles * 128;
+  a.m_valid = gated ? dm.f : dm.d;
   const int bi = bn_index(p.bn);
+  if (bi < 0) return cudaErrorInvalidValue;
   if (gated) {
     a.out = h->ws.hbuf;
     a.ld = dm.f;
     const CUtensorMap& b = h->tm_xp[bi];
+    const CUtensorMap &g = h->tm_gate, &u = h->tm_up;
     switch (p.bn) {
-      case 16: return launch_one<16, true>(h, h->tm_gate, h->tm_up, b, a, s);
-      case 32: return launch_one<32, true>(h, h->tm_gate, h->tm_up, b, a, s);
-      case 64: return launch_one<64, true>(h, h->tm_gate, h->tm_up, b, a, s);
-      case 128: return launch_one<128, true>(h, h->tm_gate, h->tm_up, b, a, s);
+      case 16: return launch_one<16, 2, true>(h, g, u, b, a, s);
+      case 32: return launch_one<32, 2, true>(h, g, u, b, a, s);
+      case 64: return launch_one<64, 2, true>(h, g, u, b, a, s);
+      case 96: return launch_one<96, 2, true>(h, g, u, b, a, s);
+      case 128: return launch_one<128, 2, true>(h, g, u, b, a, s);
+      case 160: return launch_one<160, 2, true>(h, g, u, b, a, s);
+      case 192: return launch_one<192, 2, true>(h, g, u, b, a, s);
+      case 224: return launch_one<224, 2, true>(h, g, u, b, a, s);
+      case 256: return launch_one<256, 2, true>(h, g, u, b, a, s);
       default: return cudaErrorInvalidValue;
     }
   }
   a.out = h->ws.out;
   a.ld = dm.d;
   const CUtensorMap& b = h->tm_h[bi];
+  const CUtensorMap& w = h->tm_down;
+  if (p.na == 1) {
+    switch (p.bn) {
+      case 16: return launch_one<16, 1, false>(h, w, w, b, a, s);
+      case 32: return launch_one<32, 1, false>(h, w, w, b, a, s);
+      case 64: return launch_one<64, 1, false>(h, w, w, b, a, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (p.bn) {
-    case 16: return launch_one<16, false>(h, h->tm_down, h->tm_down, b, a, s);
-    case 32: return launch_one<32, false>(h, h->tm_down, h->tm_down, b, a, s);
-    case 64: return launch_one<64, false>(h, h->tm_down, h->tm_down, b, a, s);
-    case 128: return launch_one<128, false>(h, h->tm_down, h->tm_down, b, a, s);
-    case 256: return launch_one<256, false>(h, h->tm_down, h->tm_down, b, a, s);
+    case 64: return launch_one<64, 2, false>(h, w, w, b, a, s);
+    case 96: return launch_one<96, 2, false>(h, w, w, b, a, s);
+    case 128: return launch_one<128, 2, false>(h, w, w, b, a, s);
+    case 160: return launch_one<160, 2, false>(h, w, w, b, a, s);
+    case 192: return launch_one<192, 2, false>(h, w, w, b, a, s);
+    case 224: return launch_one<224, 2, false>(h, w, w, b, a, s);
+    case 256: return launch_one<256, 2, false>(h, w, w, b, a, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -371,6 +371,7 @@ cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaSt
   a.b_k = gated ? dm.d : dm.f;
   a.m_valid = p.m_tiles * 128;
   const int bi = bn_index(p.bn);
+  if (bi < 0) return cudaErrorInvalidValue;
   if (gated) {
     a.out = h->ws.hbuf;
     a.ld = dm.f;

@@ -29,7 +29,8 @@ struct Dims {
 // One grouped GEMM launch's shape choice.
 struct GemmPlan {
   int bn;       // token rows per tile (MMA N upper bound)
-  int m_tiles;  // output features / 128
+  int na;       // weight tiles per unit (2: gate+up, or two halves of 256 features)
+  int m_tiles;  // output feature tiles (128 rows each, or 256 for a plain na = 2 unit)
   int k_blocks; // reduction / kernel K step
 };
 
@@ -78,9 +79,9 @@ struct moe_handle {
   smoe::Weights w;
   smoe::Workspace ws;
   // TMA descriptors: weights (one per projection) and the two activation
-  // matrices, the latter once per supported row-tile height (16 << i)
+  // matrices, the latter once per row-tile height 16 * (i + 1), i < 16
   CUtensorMap tm_gate, tm_up, tm_down, tm_router;
-  CUtensorMap tm_xp[5], tm_h[5];
+  CUtensorMap tm_xp[16], tm_h[16];
   int router_max_splits = 1;
   int64_t launches = 0;
   std::string last_error;
