@@ -84,6 +84,8 @@ moe_status_t fail(moe_handle* h, moe_status_t st, const std::string& msg) {
 
 moe_status_t cuda_fail(moe_handle* h, cudaError_t e, const char* what) {
   std::string m = std::string(what) + ": " + cudaGetErrorString(e);
+  if (h && !h->last_error.empty() && e == cudaErrorLaunchOutOfResources)
+    m += " (" + h->last_error + ")";  // the launcher's resource details
   if (h) h->last_error = m;
   return e == cudaErrorMemoryAllocation ? MOE_ERR_OOM : MOE_ERR_CUDA;
 }

@@ -34,13 +34,16 @@ static int pick_bn(double want, const int* cands, int n) {
   return cands[n - 1];
 }
 
-// Row-tile height: the smallest supported height >= 1.3 x the mean rows per
-// routed expert, so that nearly every expert's rows fit one tile and each
-// weight slab is read into shared memory once per forward.
+// Row-tile height: the smallest supported height >= SMOE_BN_FACTOR x the mean
+// rows per routed expert, so that nearly every expert's rows fit one tile and
+// each weight slab is read into shared memory once per forward.
+#ifndef SMOE_BN_FACTOR
+#define SMOE_BN_FACTOR 1.3  // tuning constant
+#endif
 GemmPlan plan_gate_up(const Dims& dm, int64_t T) {
   static const int bf16_bn[] = {16, 32, 64, 96, 128, 160, 192, 224, 256};
   static const int fp8_bn[] = {16, 32, 64};
-  const double want = 1.3 * static_cast<double>(T) * dm.k / dm.E;
+  const double want = SMOE_BN_FACTOR * static_cast<double>(T) * dm.k / dm.E;
   GemmPlan p;
   p.bn = dm.fp8 ? pick_bn(want, fp8_bn, 3) : pick_bn(want, bf16_bn, 9);
   p.na = 2;
@@ -54,7 +57,7 @@ GemmPlan plan_gate_up(const Dims& dm, int64_t T) {
 GemmPlan plan_down(const Dims& dm, int64_t T) {
   static const int bf16_bn[] = {16, 32, 64, 96, 128, 160, 192, 224, 256};
   static const int fp8_bn[] = {16, 32, 64, 128};
-  const double want = 1.3 * static_cast<double>(T) * dm.k / dm.E;
+  const double want = SMOE_BN_FACTOR * static_cast<double>(T) * dm.k / dm.E;
   GemmPlan p;
   p.bn = dm.fp8 ? pick_bn(want, fp8_bn, 4) : pick_bn(want, bf16_bn, 9);
   p.na = (!dm.fp8 && p.bn >= 64 && dm.d % 256 == 0) ? 2 : 1;

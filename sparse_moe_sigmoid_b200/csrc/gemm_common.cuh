@@ -40,6 +40,7 @@ struct GemmArgs {
   int b_k;                   // K extent of B; the K index into B is (k mod b_k)
   int m_valid;               // only output features < m_valid are stored
   int kpp;                   // promoted BF16 GEMM: stages accumulated in TMEM per promotion
+  int stages;                // promoted GEMM: shared-memory ring depth
 };
 
 __device__ __forceinline__ int total_units_of(const GemmArgs& a, int BN) {

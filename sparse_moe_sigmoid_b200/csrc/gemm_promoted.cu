@@ -33,8 +33,13 @@
 //
 // Roles and the bounded-wait / wind-down rules are those of the BF16 kernel
 // (gemm_bf16.cu): warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
-// warps 2..5 promotion + epilogue.
+// then NPG warpgroups of promotion + epilogue warps; group g owns columns
+// [g*BN/NPG, (g+1)*BN/NPG) of the row tile (two groups halve the promotion
+// work per thread and allow tiles of 128 rows with gate and up, 256 without).
+// The shared-memory ring's depth is set at launch from what the scale
+// staging of the actual K leaves free.
 #include <cuda_fp8.h>
+#include <stdio.h>
 
 #include "gemm_common.cuh"
 #include "internal.h"
@@ -45,46 +50,77 @@ namespace smoe {
 using namespace sm100;
 
 constexpr int kFp8MaxKBlocks = 64;  // hidden_size and moe_intermediate_size <= 8192
+constexpr int kPromMaxStages = 12;
+constexpr int kPromSmemBudget = 227 * 1024 - 2048;
 
 // FP8: e4m3 operands, 128 K per stage, block scales applied at promotion.
 // Otherwise BF16 operands, 64 K per stage, no scales.
-template <int BN, bool GATED, bool FP8>
+template <int BN, bool GATED, bool FP8, int NPG>
 struct PromCfg {
-  static constexpr int kA = 128 * 128;  // 128 rows x 128 bytes of K
+  static constexpr int kThreads = 64 + 128 * NPG;
+  static constexpr int kCols = BN / NPG;  // columns per promotion group
+  static constexpr int kA = 128 * 128;    // 128 rows x 128 bytes of K
   static constexpr int kB = BN * 128;
   static constexpr int kKPerStage = FP8 ? 128 : 64;
   static constexpr int kNumA = GATED ? 2 : 1;
   static constexpr int kStage = kA * kNumA + kB;
-  static constexpr int kScaleBytes = FP8 ? (kFp8MaxKBlocks * BN + 2 * kFp8MaxKBlocks) * 4 : 0;
   static constexpr int kAmaxBytes = GATED ? 4 * BN * 4 : 0;
-  static constexpr int kStages0 = (227 * 1024 - 2048 - kScaleBytes - kAmaxBytes) / kStage;
-  static constexpr int kStages = kStages0 > 10 ? 10 : kStages0;
   static constexpr int kPCols = GATED ? 2 * BN : BN;  // one partial buffer
   static constexpr int kTmemCols = pow2_at_least(2 * kPCols, 32);
-  static constexpr int kSmem = kStages * kStage + kScaleBytes + kAmaxBytes + 1024 + 320;
+  static constexpr int kBarrierBytes = 512;
   static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
-  static_assert(kStages >= 2, "need at least two stages");
+  static_assert(kCols % 16 == 0, "columns per group in 16-column loads");
+  static_assert((GATED ? 2 : 1) * kCols <= 64, "one promotion's loads must fit in registers");
+  static_assert(kTmemCols <= 512, "TMEM holds 512 columns");
+  static_assert(FP8 || !GATED, "the BF16 promoted GEMM is plain");
+  // scale staging of FP8: activation scales [KB][BN] and weight scales [2][KB]
+  static constexpr int scale_bytes(int kb) { return FP8 ? (kb * BN + 2 * kb) * 4 : 0; }
+  static constexpr int stages(int kb) {
+    const int n = (kPromSmemBudget - kBarrierBytes - scale_bytes(kb) - kAmaxBytes) / kStage;
+    return n > kPromMaxStages ? kPromMaxStages : n;
+  }
+  static constexpr int smem(int kb) {
+    return stages(kb) * kStage + scale_bytes(kb) + kAmaxBytes + kBarrierBytes + 1024;
+  }
 };
 
-template <int BN, bool GATED, bool FP8>
-__global__ void __launch_bounds__(192, 1)
+// registers per thread for the one CTA per SM: the register file is four
+// 16K-register slices, one per scheduler, and a block's warps are spread over
+// them, so a slice holds ceil(warps / 4) warps; rounded down to the
+// allocation granule of 8, at most 255
+template <int kThreads>
+constexpr int prom_max_regs() {
+  return (16384 / (32 * ((kThreads / 32 + 3) / 4))) / 8 * 8 > 255
+             ? 255
+             : (16384 / (32 * ((kThreads / 32 + 3) / 4))) / 8 * 8;
+}
+
+template <int NPG>
+constexpr int prom_regs() {
+  return prom_max_regs<64 + 128 * NPG>();
+}
+
+template <int BN, bool GATED, bool FP8, int NPG>
+__global__ void __maxnreg__(prom_regs<NPG>())
     grouped_gemm_promoted_kernel(const __grid_constant__ CUtensorMap tmA0,
                                  const __grid_constant__ CUtensorMap tmA1,
                                  const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
-  using C = PromCfg<BN, GATED, FP8>;
-  static_assert(FP8 || !GATED, "the BF16 promoted GEMM is plain");
+  using C = PromCfg<BN, GATED, FP8, NPG>;
+  const int KB = args.k_blocks;
+  const int S = args.stages;  // ring depth, set at launch (<= kPromMaxStages)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  float* sa_s = reinterpret_cast<float*>(smem + C::kStages * C::kStage);  // [KB][BN] (FP8)
-  float* sw_s = sa_s + (FP8 ? kFp8MaxKBlocks * BN : 0);                    // [2][KB] (FP8)
-  float* amax_s = sw_s + (FP8 ? 2 * kFp8MaxKBlocks : 0);                   // [4][BN] (gated)
-  uint64_t* full = reinterpret_cast<uint64_t*>(amax_s + (GATED ? 4 * BN : 0));
-  uint64_t* empty = full + C::kStages;
-  uint64_t* pfull = empty + C::kStages;
+  float* sa_s = reinterpret_cast<float*>(smem + S * C::kStage);  // [KB][BN] (FP8)
+  float* sw_s = sa_s + (FP8 ? KB * BN : 0);                       // [2][KB] (FP8)
+  float* amax_s = sw_s + (FP8 ? 2 * KB : 0);                      // [4][BN] (gated)
+  uint64_t* full = reinterpret_cast<uint64_t*>(
+      (reinterpret_cast<uintptr_t>(amax_s + (GATED ? 4 * BN : 0)) + 7) & ~uintptr_t(7));
+  uint64_t* empty = full + kPromMaxStages;
+  uint64_t* pfull = empty + kPromMaxStages;
   uint64_t* pempty = pfull + 2;
   uint64_t* drain = pempty + 2;
-  uint64_t* grp = drain + 1;  // the 128 promotion threads' own barrier (bounded waits)
+  uint64_t* grp = drain + 1;  // the promotion threads' own barrier (bounded waits)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(grp + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* consumed = tmem_slot + 2;
@@ -92,20 +128,19 @@ __global__ void __launch_bounds__(192, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int KB = args.k_blocks;
   const int KPP = FP8 ? 1 : args.kpp;  // stages accumulated per promotion
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&pfull[a], 1);
-      mbar_init(&pempty[a], 4);
+      mbar_init(&pempty[a], 4 * NPG);
     }
     mbar_init(drain, 1);
-    mbar_init(grp, 128);
+    mbar_init(grp, 128 * NPG);
     *abort_flag = 0;
     *consumed = 0;
     *issued = 0;
@@ -134,8 +169,8 @@ __global__ void __launch_bounds__(192, 1)
       for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
         const Unit un = decode_unit(u, args, BN);
         for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int s = it % C::kStages;
-          const uint32_t ph = (it / C::kStages) & 1u;
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1u;
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -164,8 +199,8 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t n = static_cast<uint32_t>(((un.nvalid + 15) / 16) * 16);
         const uint32_t idesc = make_idesc(FP8 ? 0u : 1u, n);
         for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int s = it % C::kStages;
-          const uint32_t ph = (it / C::kStages) & 1u;
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1u;
           const int pb = pit & 1;
           const int sub = kb % KPP;
           if ((sub == 0 && !mbar_wait(&pempty[pb], ((pit >> 1) & 1u) ^ 1u, abort_flag)) ||
@@ -205,8 +240,9 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(drain, 0, nullptr);
     }
   } else {
-    const int q = warp & 3;           // TMEM lane quarter
-    const int ptid = threadIdx.x - 64;  // 0..127 among the promotion warps
+    const int q = warp & 3;                    // TMEM lane quarter
+    const int ptid = threadIdx.x - 64;         // 0 .. 128*NPG-1 among the promotion warps
+    const int c_begin = (ptid >> 7) * C::kCols;  // this group's first column
     uint32_t pit = 0, gph = 0;
     bool ok = true;
     auto group_sync = [&]() {
@@ -224,14 +260,14 @@ __global__ void __launch_bounds__(192, 1)
           ok = false;
           break;
         }
-        for (int i = ptid; i < KB * BN; i += 128) {
+        for (int i = ptid; i < KB * BN; i += 128 * NPG) {
           const int kb = i / BN, j = i - kb * BN;
           sa_s[i] = j < un.nvalid ? __ldg(args.act_scale + (size_t)(un.row0 + j) * KB + kb) : 0.f;
         }
         const size_t wrow = ((size_t)un.g * args.m_tiles + un.mt) * KB;
-        for (int i = ptid; i < KB; i += 128) {
+        for (int i = ptid; i < KB; i += 128 * NPG) {
           sw_s[i] = __ldg(args.w_scale0 + wrow + i);
-          if (GATED) sw_s[kFp8MaxKBlocks + i] = __ldg(args.w_scale1 + wrow + i);
+          if (GATED) sw_s[KB + i] = __ldg(args.w_scale1 + wrow + i);
         }
         if (!group_sync()) {
           ok = false;
@@ -239,9 +275,9 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
 
-      float acc0[BN], acc1[GATED ? BN : 1];
+      float acc0[C::kCols], acc1[GATED ? C::kCols : 1];
 #pragma unroll
-      for (int j = 0; j < BN; ++j) {
+      for (int j = 0; j < C::kCols; ++j) {
         acc0[j] = 0.f;
         if (GATED) acc1[j] = 0.f;
       }
@@ -254,24 +290,34 @@ __global__ void __launch_bounds__(192, 1)
         }
         tc_fence_after();
         const float sw0 = FP8 ? sw_s[pg] : 1.f;
-        const float sw1 = (FP8 && GATED) ? sw_s[kFp8MaxKBlocks + pg] : 0.f;
-        const float* sa = sa_s + pg * BN;
+        const float sw1 = (FP8 && GATED) ? sw_s[KB + pg] : 0.f;
+        const float* sa = sa_s + pg * BN + c_begin;
+        // every load first, one wait, then the arithmetic: tcgen05.wait::ld
+        // waits for all outstanding loads, so a wait per chunk would pay the
+        // TMEM round trip once per chunk
+        uint32_t g[C::kCols], v[GATED ? C::kCols : 1];
 #pragma unroll
-        for (int c = 0; c < BN / 16; ++c) {
-          if (c * 16 < un.nvalid) {
-            uint32_t g[16], v[16];
-            tmem_ld16(tq + pb * C::kPCols + c * 16, g);
-            if (GATED) tmem_ld16(tq + pb * C::kPCols + BN + c * 16, v);
-            tmem_ld_wait();
+        for (int c = 0; c < C::kCols / 16; ++c) {
+          if (c_begin + c * 16 < un.nvalid) {
+            tmem_ld16(tq + pb * C::kPCols + c_begin + c * 16,
+                      *reinterpret_cast<uint32_t(*)[16]>(&g[c * 16]));
+            if (GATED)
+              tmem_ld16(tq + pb * C::kPCols + BN + c_begin + c * 16,
+                        *reinterpret_cast<uint32_t(*)[16]>(&v[c * 16]));
+          }
+        }
+        tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
+        for (int c = 0; c < C::kCols / 16; ++c) {
+          if (c_begin + c * 16 < un.nvalid) {
+#pragma unroll
+            for (int j = c * 16; j < c * 16 + 16; ++j) {
               if (FP8) {
-                const float s = sa[c * 16 + j];
-                acc0[c * 16 + j] = fmaf(__uint_as_float(g[j]), sw0 * s, acc0[c * 16 + j]);
-                if (GATED)
-                  acc1[c * 16 + j] = fmaf(__uint_as_float(v[j]), sw1 * s, acc1[c * 16 + j]);
+                const float s = sa[j];
+                acc0[j] = fmaf(__uint_as_float(g[j]), sw0 * s, acc0[j]);
+                if (GATED) acc1[j] = fmaf(__uint_as_float(v[j]), sw1 * s, acc1[j]);
               } else {
-                acc0[c * 16 + j] += __uint_as_float(g[j]);
+                acc0[j] += __uint_as_float(g[j]);
               }
             }
           }
@@ -287,12 +333,12 @@ __global__ void __launch_bounds__(192, 1)
         // h = silu(g) * u, then per-row e4m3 quantisation over this tile's 128 features
         uint8_t* hq = static_cast<uint8_t*>(args.out);
 #pragma unroll
-        for (int j = 0; j < BN; ++j) {
+        for (int j = 0; j < C::kCols; ++j) {
           const float gv = acc0[j];
           acc0[j] = gv / (1.f + expf(-gv)) * acc1[j];
-          if (j < un.nvalid) {
+          if (c_begin + j < un.nvalid) {
             const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(acc0[j])));
-            if (lane == 0) amax_s[q * BN + j] = __uint_as_float(m);
+            if (lane == 0) amax_s[q * BN + c_begin + j] = __uint_as_float(m);
           }
         }
         if (!group_sync()) {
@@ -300,26 +346,28 @@ __global__ void __launch_bounds__(192, 1)
           break;
         }
 #pragma unroll
-        for (int j = 0; j < BN; ++j) {
-          if (j < un.nvalid) {
-            const float amax = fmaxf(fmaxf(amax_s[j], amax_s[BN + j]),
-                                     fmaxf(amax_s[2 * BN + j], amax_s[3 * BN + j]));
+        for (int j = 0; j < C::kCols; ++j) {
+          const int col = c_begin + j;
+          if (col < un.nvalid) {
+            const float amax = fmaxf(fmaxf(amax_s[col], amax_s[BN + col]),
+                                     fmaxf(amax_s[2 * BN + col], amax_s[3 * BN + col]));
             const float sh = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-            const size_t row = static_cast<size_t>(un.row0 + j);
+            const size_t row = static_cast<size_t>(un.row0 + col);
             float2 pair;
             pair.x = __fdiv_rn(acc0[j], sh);
             pair.y = 0.f;
             const __nv_fp8x2_storage_t b = __nv_cvt_float2_to_fp8x2(pair, __NV_SATFINITE, __NV_E4M3);
             hq[row * args.ld + feat] = static_cast<uint8_t>(b & 0xFF);
-            if (ptid == 0) args.out_scale[row * args.m_tiles + un.mt] = sh;
+            if (q == 0 && lane == 0) args.out_scale[row * args.m_tiles + un.mt] = sh;
           }
         }
       } else {
         float* out = static_cast<float*>(args.out);
         if (feat < args.m_valid) {
 #pragma unroll
-          for (int j = 0; j < BN; ++j)
-            if (j < un.nvalid) out[static_cast<size_t>(un.row0 + j) * args.ld + feat] = acc0[j];
+          for (int j = 0; j < C::kCols; ++j)
+            if (c_begin + j < un.nvalid)
+              out[static_cast<size_t>(un.row0 + c_begin + j) * args.ld + feat] = acc0[j];
         }
       }
     }
@@ -334,27 +382,43 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   if (*abort_flag && warp == 0 && lane == 0) {
     for (uint32_t j = *consumed; j < *issued; ++j)
-      mbar_wait(&full[j % C::kStages], (j / C::kStages) & 1u, nullptr);
+      mbar_wait(&full[j % S], (j / S) & 1u, nullptr);
   }
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
-template <int BN, bool GATED, bool FP8 = true>
+template <int BN, bool GATED, bool FP8, int NPG>
 static cudaError_t launch_one(moe_handle* h, const CUtensorMap& a0, const CUtensorMap& a1,
-                              const CUtensorMap& b, const GemmArgs& args, cudaStream_t s) {
-  using C = PromCfg<BN, GATED, FP8>;
+                              const CUtensorMap& b, GemmArgs args, cudaStream_t s) {
+  using C = PromCfg<BN, GATED, FP8, NPG>;
   static bool configured[64] = {};
   if (h->device < 64 && !configured[h->device]) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_promoted_kernel<BN, GATED, FP8>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_promoted_kernel<BN, GATED, FP8, NPG>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kPromSmemBudget + 1024);
     if (e != cudaSuccess) return e;
     configured[h->device] = true;
   }
-  grouped_gemm_promoted_kernel<BN, GATED, FP8><<<h->num_sms, 192, C::kSmem, s>>>(a0, a1, b, args);
+  args.stages = C::stages(args.k_blocks);
+  if (args.stages < 2) return cudaErrorInvalidValue;
+  const int smem = C::smem(args.k_blocks);
+  grouped_gemm_promoted_kernel<BN, GATED, FP8, NPG><<<h->num_sms, C::kThreads, smem, s>>>(
+      a0, a1, b, args);
   h->launches++;
-  return cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaErrorLaunchOutOfResources) {
+    cudaFuncAttributes fa{};
+    cudaFuncGetAttributes(&fa, grouped_gemm_promoted_kernel<BN, GATED, FP8, NPG>);
+    char buf[256];
+    snprintf(buf, sizeof buf,
+             "promoted GEMM BN=%d: %d threads x %d registers, %zu B local, max threads %d, "
+             "%d B dynamic smem",
+             BN, C::kThreads, fa.numRegs, fa.localSizeBytes, fa.maxThreadsPerBlock, smem);
+    h->last_error = buf;
+  }
+  return e;
 }
 
 cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaStream_t s) {
@@ -380,10 +444,11 @@ cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaSt
     a.w_scale1 = h->w.up_s;
     a.act_scale = h->ws.xs;
     const CUtensorMap& b = h->tm_xp[bi];
+    const CUtensorMap &g = h->tm_gate, &u = h->tm_up;
     switch (p.bn) {
-      case 16: return launch_one<16, true>(h, h->tm_gate, h->tm_up, b, a, s);
-      case 32: return launch_one<32, true>(h, h->tm_gate, h->tm_up, b, a, s);
-      case 64: return launch_one<64, true>(h, h->tm_gate, h->tm_up, b, a, s);
+      case 16: return launch_one<16, true, true, 1>(h, g, u, b, a, s);
+      case 32: return launch_one<32, true, true, 1>(h, g, u, b, a, s);
+      case 64: return launch_one<64, true, true, 2>(h, g, u, b, a, s);
       default: return cudaErrorInvalidValue;
     }
   }
@@ -393,11 +458,12 @@ cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaSt
   a.w_scale1 = h->w.down_s;
   a.act_scale = h->ws.hs;
   const CUtensorMap& b = h->tm_h[bi];
+  const CUtensorMap& w = h->tm_down;
   switch (p.bn) {
-    case 16: return launch_one<16, false>(h, h->tm_down, h->tm_down, b, a, s);
-    case 32: return launch_one<32, false>(h, h->tm_down, h->tm_down, b, a, s);
-    case 64: return launch_one<64, false>(h, h->tm_down, h->tm_down, b, a, s);
-    case 128: return launch_one<128, false>(h, h->tm_down, h->tm_down, b, a, s);
+    case 16: return launch_one<16, false, true, 1>(h, w, w, b, a, s);
+    case 32: return launch_one<32, false, true, 1>(h, w, w, b, a, s);
+    case 64: return launch_one<64, false, true, 1>(h, w, w, b, a, s);
+    case 128: return launch_one<128, false, true, 2>(h, w, w, b, a, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -435,7 +501,7 @@ cudaError_t launch_router_gemm(moe_handle* h, const void* x, int T, cudaStream_t
   a.out = h->ws.logits_part;
   a.ld = dm.E;
   a.status = h->ws.status;
-  return launch_one<BN, false, false>(h, h->tm_router, h->tm_router, tmx, a, s);
+  return launch_one<BN, false, false, 2>(h, h->tm_router, h->tm_router, tmx, a, s);
 }
 
 }  // namespace smoe
