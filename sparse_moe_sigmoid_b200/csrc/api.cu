@@ -457,12 +457,16 @@ moe_status_t moe_forward(moe_handle_t* h, const void* x, int64_t T, void* y,
   mark(4);
   if (dm.fp8) {
     CUDA_TRY(h, smoe::launch_gemm_fp8(h, true, p1, s), "gate/up GEMM launch");
+  } else if (p1.pair) {
+    CUDA_TRY(h, smoe::launch_gemm_bf16_pair(h, true, p1, s), "gate/up GEMM launch");
   } else {
     CUDA_TRY(h, smoe::launch_gemm_bf16(h, true, p1, s), "gate/up GEMM launch");
   }
   mark(5);
   if (dm.fp8) {
     CUDA_TRY(h, smoe::launch_gemm_fp8(h, false, p2, s), "down GEMM launch");
+  } else if (p2.pair) {
+    CUDA_TRY(h, smoe::launch_gemm_bf16_pair(h, false, p2, s), "down GEMM launch");
   } else {
     CUDA_TRY(h, smoe::launch_gemm_bf16(h, false, p2, s), "down GEMM launch");
   }

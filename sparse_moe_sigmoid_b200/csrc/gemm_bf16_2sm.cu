@@ -1,0 +1,321 @@
+// Grouped expert GEMMs (BF16) on CTA pairs: the same computation as
+// gemm_bf16.cu for tall row tiles, with the 2-SM tensor-core MMA.
+//
+// One tcgen05.mma is issued by one thread, and a thread issues one every
+// ~50-80 cycles; an M = 128 MMA with N = 176 rows holds ~88 cycles of tensor
+// work, so a single CTA barely keeps its tensor core fed. The pair MMA
+// (cta_group::2, M = 256) does twice the work per issued instruction: each
+// CTA of a cluster pair holds 128 weight rows and half of the row tile in its
+// own shared memory, and each CTA's TMEM receives its 128 rows of the result.
+//
+// A unit is (expert, 256 output features, row tile). Per CTA pair:
+//   producers (warp 0 of each CTA) load that CTA's weight rows (gate and up,
+//     or the down projection's) and its half of the row tile; both count
+//     their bytes on the even CTA's `full` barrier;
+//   the even CTA's warp 1 issues the pair MMAs and commits to the `empty`
+//     barriers of both CTAs (and, per unit, to both `tfull` barriers);
+//   each CTA's epilogue warps drain their own TMEM (SwiGLU + BF16 h, or the
+//     fp32 per-row output) and signal the even CTA's `tempty` barrier.
+// Every wait is bounded as in gemm_bf16.cu. The only unbounded step is the
+// cluster barrier at entry and exit, which both CTAs always reach.
+#include <cuda_bf16.h>
+#include <stdio.h>
+
+#include "gemm_common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace smoe {
+
+using namespace sm100;
+
+template <int BN, bool SWIGLU>
+struct Pair2Cfg {
+  static constexpr int kA = 128 * 64 * 2;        // this CTA's 128 x 64 BF16 weight tile
+  static constexpr int kB = (BN / 2) * 64 * 2;   // this CTA's half of the row tile
+  static constexpr int kNumA = SWIGLU ? 2 : 1;
+  static constexpr int kStage = kA * kNumA + kB;
+  static constexpr int kStages0 = (227 * 1024 - 2048) / kStage;
+  static constexpr int kStages = kStages0 > 12 ? 12 : kStages0;
+  static constexpr int kAccCols = kNumA * BN;
+  static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
+  static constexpr int kTmemCols = pow2_at_least(kAccBufs * kAccCols, 32);
+  static constexpr int kSmem = kStages * kStage + 1024 + 256;
+  static_assert(BN % 32 == 0, "each CTA's half of the row tile is a multiple of 16 rows");
+  static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
+  static_assert(kTmemCols <= 512, "TMEM holds 512 columns");
+  static_assert(kStages >= 2, "need at least two stages");
+};
+
+template <int BN, bool SWIGLU>
+__global__ void __launch_bounds__(192, 1)
+    grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA0,
+                                  const __grid_constant__ CUtensorMap tmA1,
+                                  const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+  using C = Pair2Cfg<BN, SWIGLU>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStage);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  volatile uint32_t* consumed = tmem_slot + 2;
+  volatile uint32_t* issued = tmem_slot + 3;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < C::kAccBufs; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 8);  // four epilogue warps in each CTA
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *consumed = 0;
+    *issued = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA0);
+    if (SWIGLU) tma_prefetch_desc(&tmA1);
+    tma_prefetch_desc(&tmB);
+  }
+  cluster_sync();  // the peer's barriers exist before anything signals them
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, C::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' TMEM is allocated before the first pair MMA
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total_units = total_units_of(args, BN);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int u = pair; u < total_units && ok; u += npairs) {
+        const Unit un = decode_unit(u, args, BN);
+        const int n = ((un.nvalid + 31) / 32) * 32;  // MMA N: halves of 16-row multiples
+        const int arow = un.mt * 256 + static_cast<int>(rank) * 128;
+        const int brow = un.row0 + static_cast<int>(rank) * (n / 2);
+        for (int kb = 0; kb < args.k_blocks; ++kb, ++it) {
+          const int s = it % C::kStages;
+          const uint32_t ph = (it / C::kStages) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * C::kStage;
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::kStage);
+          tma_load_3d_pair(st, &tmA0, &full[s], kb * 64, arow, un.g);
+          if (SWIGLU) tma_load_3d_pair(st + C::kA, &tmA1, &full[s], kb * 64, arow, un.g);
+          tma_load_2d_pair(st + C::kA * C::kNumA, &tmB, &full[s], kb * 64, brow);
+          *issued = it + 1;
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(args.status, MOE_DEVICE_WAIT_TIMEOUT);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      int i = 0;
+      for (int u = pair; u < total_units && ok; u += npairs, ++i) {
+        const Unit un = decode_unit(u, args, BN);
+        const int acc = i % C::kAccBufs;
+        const int use = i / C::kAccBufs;
+        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + acc * C::kAccCols;
+        const uint32_t n = static_cast<uint32_t>(((un.nvalid + 31) / 32) * 32);
+        const uint32_t idesc = make_idesc(1u, n, 256);
+        for (int kb = 0; kb < args.k_blocks; ++kb, ++it) {
+          const int s = it % C::kStages;
+          const uint32_t ph = (it / C::kStages) & 1u;
+          if (!mbar_wait(&full[s], ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + s * C::kStage);
+          const uint64_t ad0 = sw128_kmajor_desc(a0);
+          const uint64_t ad1 = sw128_kmajor_desc(a0 + C::kA);
+          const uint64_t bd = sw128_kmajor_desc(a0 + C::kA * C::kNumA);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t accum = (kb | k) ? 1u : 0u;
+            mma_bf16_pair(d0, ad0 + 2 * k, bd + 2 * k, idesc, accum);
+            if (SWIGLU) mma_bf16_pair(d0 + BN, ad1 + 2 * k, bd + 2 * k, idesc, accum);
+          }
+          mma_commit_pair(&empty[s], 0x3);
+          *consumed = it + 1;
+        }
+        if (!ok) break;
+        mma_commit_pair(&tfull[acc], 0x3);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(args.status, MOE_DEVICE_WAIT_TIMEOUT);
+      }
+      mma_commit_pair(drain, 0x1);  // this CTA only
+      mbar_wait(drain, 0, nullptr);
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int i = 0;
+    for (int u = pair; u < total_units; u += npairs, ++i) {
+      const Unit un = decode_unit(u, args, BN);
+      const int acc = i % C::kAccBufs;
+      const int use = i / C::kAccBufs;
+      if (!mbar_wait(&tfull[acc], use & 1, abort_flag)) {
+        if (lane == 0) {
+          *abort_flag = 1;
+          atomicOr(args.status, MOE_DEVICE_WAIT_TIMEOUT);
+        }
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::kAccCols;
+      const int feat = un.mt * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
+      for (int c0 = 0; c0 < un.nvalid; c0 += 16) {
+        uint32_t g[16], v[16];
+        tmem_ld16(tb + c0, g);
+        if (SWIGLU) tmem_ld16(tb + BN + c0, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int col = c0 + j;
+          if (col < un.nvalid) {
+            const size_t row = static_cast<size_t>(un.row0 + col);
+            if (SWIGLU) {
+              const float gv = __uint_as_float(g[j]);
+              const float uv = __uint_as_float(v[j]);
+              const float hv = gv / (1.f + expf(-gv)) * uv;
+              static_cast<__nv_bfloat16*>(args.out)[row * args.ld + feat] = __float2bfloat16_rn(hv);
+            } else if (feat < args.m_valid) {
+              static_cast<float*>(args.out)[row * args.ld + feat] = __uint_as_float(g[j]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0) mbar_arrive(&tempty[acc]);
+        else mbar_arrive_remote(&tempty[acc], 0);
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && rank == 0 && warp == 0 && lane == 0) {
+    // loads counted on this CTA's full barriers (both CTAs') that were never
+    // consumed: let them land before either CTA exits
+    for (uint32_t j = *consumed; j < *issued; ++j)
+      mbar_wait(&full[j % C::kStages], (j / C::kStages) & 1u, nullptr);
+  }
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, C::kTmemCols);
+}
+
+template <int BN, bool SWIGLU>
+static cudaError_t launch_pair(moe_handle* h, const CUtensorMap& a0, const CUtensorMap& a1,
+                               const CUtensorMap& b, const GemmArgs& args, cudaStream_t s) {
+  using C = Pair2Cfg<BN, SWIGLU>;
+  auto kern = grouped_gemm_bf16_pair_kernel<BN, SWIGLU>;
+  static bool configured[64] = {};
+  if (h->device < 64 && !configured[h->device]) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (e != cudaSuccess) return e;
+    configured[h->device] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(h->num_sms & ~1));
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a0, a1, b, args);
+  h->launches++;
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+// The pair kernel's row-tile heights (multiples of 32, each CTA taking half).
+bool pair_bn_supported(int bn) {
+  return bn == 128 || bn == 160 || bn == 192 || bn == 224 || bn == 256;
+}
+
+cudaError_t launch_gemm_bf16_pair(moe_handle* h, bool gated, const GemmPlan& p, cudaStream_t s) {
+  const Dims& dm = h->dims;
+  GemmArgs a{};
+  a.offsets = h->ws.offsets;
+  a.unit_base = h->ws.unit_base + (gated ? 0 : (dm.G + 1));
+  a.G = dm.G;
+  a.m_tiles = p.m_tiles;
+  a.k_blocks = p.k_blocks;
+  a.bn = p.bn;
+  a.status = h->ws.status;
+  a.b_k = gated ? dm.d : dm.f;
+  a.m_valid = gated ? dm.f : dm.d;
+  const int bi = bn_index(p.bn / 2);  // each CTA's B box is half the row tile
+  if (bi < 0) return cudaErrorInvalidValue;
+  if (gated) {
+    a.out = h->ws.hbuf;
+    a.ld = dm.f;
+    const CUtensorMap& b = h->tm_xp[bi];
+    const CUtensorMap &g = h->tm_gate, &u = h->tm_up;
+    switch (p.bn) {
+      case 128: return launch_pair<128, true>(h, g, u, b, a, s);
+      case 160: return launch_pair<160, true>(h, g, u, b, a, s);
+      case 192: return launch_pair<192, true>(h, g, u, b, a, s);
+      case 224: return launch_pair<224, true>(h, g, u, b, a, s);
+      case 256: return launch_pair<256, true>(h, g, u, b, a, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  a.out = h->ws.out;
+  a.ld = dm.d;
+  const CUtensorMap& b = h->tm_h[bi];
+  const CUtensorMap& w = h->tm_down;
+  switch (p.bn) {
+    case 128: return launch_pair<128, false>(h, w, w, b, a, s);
+    case 160: return launch_pair<160, false>(h, w, w, b, a, s);
+    case 192: return launch_pair<192, false>(h, w, w, b, a, s);
+    case 224: return launch_pair<224, false>(h, w, w, b, a, s);
+    case 256: return launch_pair<256, false>(h, w, w, b, a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace smoe

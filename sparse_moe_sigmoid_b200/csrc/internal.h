@@ -30,6 +30,7 @@ struct Dims {
 struct GemmPlan {
   int bn;       // token rows per tile (MMA N upper bound)
   int na;       // weight tiles per unit (2: gate+up, or two halves of 256 features)
+  bool pair;    // BF16 on CTA pairs (2-SM MMA): units of 256 output features
   int m_tiles;  // output feature tiles (128 rows each, or 256 for a plain na = 2 unit)
   int k_blocks; // reduction / kernel K step
 };
@@ -117,6 +118,8 @@ cudaError_t launch_act_quant(const void* x, int64_t rows, int d, uint8_t* q, flo
                              cudaStream_t st);
 // gemm_bf16.cu / gemm_promoted.cu
 cudaError_t launch_gemm_bf16(moe_handle* h, bool gated, const GemmPlan& p, cudaStream_t s);
+cudaError_t launch_gemm_bf16_pair(moe_handle* h, bool gated, const GemmPlan& p, cudaStream_t s);
+bool pair_bn_supported(int bn);
 cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaStream_t s);
 int bn_index(int bn);
 // api.cu
