@@ -38,7 +38,7 @@ static int pick_bn(double want, const int* cands, int n) {
 // rows per routed expert, so that nearly every expert's rows fit one tile and
 // each weight slab is read into shared memory once per forward.
 #ifndef SMOE_BN_FACTOR
-#define SMOE_BN_FACTOR 1.3  // tuning constant
+#define SMOE_BN_FACTOR 1.5  // tuning constant
 #endif
 GemmPlan plan_gate_up(const Dims& dm, int64_t T) {
   static const int bf16_bn[] = {16, 32, 64, 96, 128, 160, 192, 224, 256};

@@ -14,8 +14,17 @@
 //     their bytes on the even CTA's `full` barrier;
 //   the even CTA's warp 1 issues the pair MMAs and commits to the `empty`
 //     barriers of both CTAs (and, per unit, to both `tfull` barriers);
-//   each CTA's epilogue warps drain their own TMEM (SwiGLU + BF16 h, or the
-//     fp32 per-row output) and signal the even CTA's `tempty` barrier.
+//   each CTA's eight epilogue warps (two per TMEM lane quarter, taking
+//     alternate 16-column chunks) drain their own TMEM (SwiGLU + BF16 h, or
+//     the fp32 per-row output) and signal the even CTA's `tempty` barrier.
+//
+// Shared-memory fill from L2, not the tensor core, bounds these kernels at
+// prefill sizes (measured: as fast with the MMAs removed), so each unit loads
+// only the activation rows its MMA reads: one tensor map per box height (16,
+// 32, ..., 128 rows per CTA), picked from the unit's row count. When the
+// gated accumulators fill TMEM (row tiles over 128, one buffer), the epilogue
+// computes h into packed BF16 registers, releases TMEM, and only then stores,
+// so the next unit's MMAs overlap the global stores.
 // Every wait is bounded as in gemm_bf16.cu. The only unbounded step is the
 // cluster barrier at entry and exit, which both CTAs always reach.
 #include <cuda_bf16.h>
@@ -28,6 +37,17 @@
 namespace smoe {
 
 using namespace sm100;
+
+constexpr int kPairBoxes = 8;     // activation box heights 16, 32, ..., 128 rows
+constexpr int kPairEpiWarps = 8;  // two per TMEM lane quarter
+constexpr int kPairThreads = 64 + 32 * kPairEpiWarps;
+// The register file is four 16K-register slices, one per SM sub-partition,
+// and warp w runs on slice w % 4: ten warps put three on a slice.
+constexpr int kPairRegs = 16384 / (32 * ((kPairThreads / 32 + 3) / 4)) / 8 * 8;
+
+struct PairBoxMaps {
+  CUtensorMap m[kPairBoxes];  // m[i]: box of 16 * (i + 1) rows x 64 columns
+};
 
 template <int BN, bool SWIGLU>
 struct Pair2Cfg {
@@ -45,13 +65,27 @@ struct Pair2Cfg {
   static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(kTmemCols <= 512, "TMEM holds 512 columns");
   static_assert(kStages >= 2, "need at least two stages");
+  static_assert(BN / 2 <= 16 * kPairBoxes, "a box per half row tile");
+  // gated tiles that fill TMEM drain into registers first (two BF16 per
+  // register, half of the 16-column chunks per warp)
+  static constexpr bool kDrainFirst = SWIGLU && kAccBufs == 1;
+  static constexpr int kChunksPerWarp = BN / 32;
 };
 
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  return __fdividef(g, 1.f + __expf(-g)) * u;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
 template <int BN, bool SWIGLU>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __maxnreg__(kPairRegs)
     grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA0,
                                   const __grid_constant__ CUtensorMap tmA1,
-                                  const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+                                  const __grid_constant__ PairBoxMaps tmB, const GemmArgs args) {
   using C = Pair2Cfg<BN, SWIGLU>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -79,7 +113,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < C::kAccBufs; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 8);  // four epilogue warps in each CTA
+      mbar_init(&tempty[a], 2 * kPairEpiWarps);  // the epilogue warps of both CTAs
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -88,10 +122,10 @@ __global__ void __launch_bounds__(192, 1)
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA0);
-    if (SWIGLU) tma_prefetch_desc(&tmA1);
-    tma_prefetch_desc(&tmB);
+  if (warp == 0) {
+    if (lane == 0) tma_prefetch_desc(&tmA0);
+    if (SWIGLU && lane == 1) tma_prefetch_desc(&tmA1);
+    if (lane >= 2 && lane - 2 < BN / 32) tma_prefetch_desc(&tmB.m[lane - 2]);
   }
   cluster_sync();  // the peer's barriers exist before anything signals them
   if (warp == 1) {
@@ -113,6 +147,8 @@ __global__ void __launch_bounds__(192, 1)
         const int n = ((un.nvalid + 31) / 32) * 32;  // MMA N: halves of 16-row multiples
         const int arow = un.mt * 256 + static_cast<int>(rank) * 128;
         const int brow = un.row0 + static_cast<int>(rank) * (n / 2);
+        const CUtensorMap* bmap = &tmB.m[n / 32 - 1];  // box of n / 2 rows
+        const uint32_t tx = 2u * static_cast<uint32_t>(C::kA * C::kNumA + (n / 2) * 128);
         for (int kb = 0; kb < args.k_blocks; ++kb, ++it) {
           const int s = it % C::kStages;
           const uint32_t ph = (it / C::kStages) & 1u;
@@ -121,10 +157,10 @@ __global__ void __launch_bounds__(192, 1)
             break;
           }
           uint8_t* st = smem + s * C::kStage;
-          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::kStage);
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], tx);
           tma_load_3d_pair(st, &tmA0, &full[s], kb * 64, arow, un.g);
           if (SWIGLU) tma_load_3d_pair(st + C::kA, &tmA1, &full[s], kb * 64, arow, un.g);
-          tma_load_2d_pair(st + C::kA * C::kNumA, &tmB, &full[s], kb * 64, brow);
+          tma_load_2d_pair(st + C::kA * C::kNumA, bmap, &full[s], kb * 64, brow);
           *issued = it + 1;
         }
       }
@@ -182,7 +218,8 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(drain, 0, nullptr);
     }
   } else {
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;           // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;  // which alternate 16-column chunks
     int i = 0;
     for (int u = pair; u < total_units; u += npairs, ++i) {
       const Unit un = decode_unit(u, args, BN);
@@ -198,32 +235,69 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::kAccCols;
       const int feat = un.mt * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
-      for (int c0 = 0; c0 < un.nvalid; c0 += 16) {
-        uint32_t g[16], v[16];
-        tmem_ld16(tb + c0, g);
-        if (SWIGLU) tmem_ld16(tb + BN + c0, v);
-        tmem_ld_wait();
+      if constexpr (C::kDrainFirst) {
+        uint32_t hp[C::kChunksPerWarp * 8];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int col = c0 + j;
-          if (col < un.nvalid) {
-            const size_t row = static_cast<size_t>(un.row0 + col);
-            if (SWIGLU) {
-              const float gv = __uint_as_float(g[j]);
-              const float uv = __uint_as_float(v[j]);
-              const float hv = gv / (1.f + expf(-gv)) * uv;
-              static_cast<__nv_bfloat16*>(args.out)[row * args.ld + feat] = __float2bfloat16_rn(hv);
-            } else if (feat < args.m_valid) {
-              static_cast<float*>(args.out)[row * args.ld + feat] = __uint_as_float(g[j]);
+        for (int j = 0; j < C::kChunksPerWarp; ++j) {
+          const int c0 = (2 * j + half) * 16;
+          if (c0 < un.nvalid) {
+            uint32_t g[16], v[16];
+            tmem_ld16(tb + c0, g);
+            tmem_ld16(tb + BN + c0, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              hp[j * 8 + e] =
+                  pack_bf16x2(silu_mul(__uint_as_float(g[2 * e]), __uint_as_float(v[2 * e])),
+                              silu_mul(__uint_as_float(g[2 * e + 1]), __uint_as_float(v[2 * e + 1])));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0) mbar_arrive(&tempty[acc]);
+          else mbar_arrive_remote(&tempty[acc], 0);
+        }
+        uint16_t* out = static_cast<uint16_t*>(args.out);
+#pragma unroll
+        for (int j = 0; j < C::kChunksPerWarp; ++j) {
+          const int c0 = (2 * j + half) * 16;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int col = c0 + e;
+            if (col < un.nvalid) {
+              const uint32_t w = hp[j * 8 + e / 2];
+              out[static_cast<size_t>(un.row0 + col) * args.ld + feat] =
+                  static_cast<uint16_t>((e & 1) ? (w >> 16) : (w & 0xFFFFu));
             }
           }
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (rank == 0) mbar_arrive(&tempty[acc]);
-        else mbar_arrive_remote(&tempty[acc], 0);
+      } else {
+        for (int c0 = half * 16; c0 < un.nvalid; c0 += 32) {
+          uint32_t g[16], v[16];
+          tmem_ld16(tb + c0, g);
+          if (SWIGLU) tmem_ld16(tb + BN + c0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int col = c0 + j;
+            if (col < un.nvalid) {
+              const size_t row = static_cast<size_t>(un.row0 + col);
+              if (SWIGLU) {
+                const float hv = silu_mul(__uint_as_float(g[j]), __uint_as_float(v[j]));
+                static_cast<__nv_bfloat16*>(args.out)[row * args.ld + feat] = __float2bfloat16_rn(hv);
+              } else if (feat < args.m_valid) {
+                static_cast<float*>(args.out)[row * args.ld + feat] = __uint_as_float(g[j]);
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0) mbar_arrive(&tempty[acc]);
+          else mbar_arrive_remote(&tempty[acc], 0);
+        }
       }
     }
   }
@@ -244,7 +318,7 @@ __global__ void __launch_bounds__(192, 1)
 
 template <int BN, bool SWIGLU>
 static cudaError_t launch_pair(moe_handle* h, const CUtensorMap& a0, const CUtensorMap& a1,
-                               const CUtensorMap& b, const GemmArgs& args, cudaStream_t s) {
+                               const PairBoxMaps& b, const GemmArgs& args, cudaStream_t s) {
   using C = Pair2Cfg<BN, SWIGLU>;
   auto kern = grouped_gemm_bf16_pair_kernel<BN, SWIGLU>;
   static bool configured[64] = {};
@@ -256,7 +330,7 @@ static cudaError_t launch_pair(moe_handle* h, const CUtensorMap& a0, const CUten
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(h->num_sms & ~1));
-  cfg.blockDim = dim3(192);
+  cfg.blockDim = dim3(kPairThreads);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -288,12 +362,13 @@ cudaError_t launch_gemm_bf16_pair(moe_handle* h, bool gated, const GemmPlan& p, 
   a.status = h->ws.status;
   a.b_k = gated ? dm.d : dm.f;
   a.m_valid = gated ? dm.f : dm.d;
-  const int bi = bn_index(p.bn / 2);  // each CTA's B box is half the row tile
-  if (bi < 0) return cudaErrorInvalidValue;
+  // activation maps with boxes of 16, 32, ..., 128 rows (each CTA's half of
+  // a row tile of 32, 64, ..., 256)
+  PairBoxMaps b;
+  for (int i = 0; i < kPairBoxes; ++i) b.m[i] = (gated ? h->tm_xp : h->tm_h)[bn_index(16 * (i + 1))];
   if (gated) {
     a.out = h->ws.hbuf;
     a.ld = dm.f;
-    const CUtensorMap& b = h->tm_xp[bi];
     const CUtensorMap &g = h->tm_gate, &u = h->tm_up;
     switch (p.bn) {
       case 128: return launch_pair<128, true>(h, g, u, b, a, s);
@@ -306,7 +381,6 @@ cudaError_t launch_gemm_bf16_pair(moe_handle* h, bool gated, const GemmPlan& p, 
   }
   a.out = h->ws.out;
   a.ld = dm.d;
-  const CUtensorMap& b = h->tm_h[bi];
   const CUtensorMap& w = h->tm_down;
   switch (p.bn) {
     case 128: return launch_pair<128, false>(h, w, w, b, a, s);
