@@ -62,7 +62,7 @@ GemmPlan plan_down(const Dims& dm, int64_t T) {
   const double want = SMOE_BN_FACTOR * static_cast<double>(T) * dm.k / dm.E;
   GemmPlan p;
   p.bn = dm.fp8 ? pick_bn(want, fp8_bn, 4) : pick_bn(want, bf16_bn, 9);
-  p.pair = !dm.fp8 && pair_bn_supported(p.bn) && dm.d % 256 == 0;
+  p.pair = !dm.fp8 && pair_bn_supported(p.bn) && dm.d % 256 == 0 && dm.f % 128 == 0;
   p.na = (!dm.fp8 && !p.pair && p.bn >= 64 && dm.d % 256 == 0) ? 2 : 1;
   p.m_tiles = dm.d / (p.pair ? 256 : kBlock * p.na);
   p.k_blocks = dm.fp8 ? dm.f / 128 : dm.f / 64;

@@ -54,7 +54,12 @@ struct Pair2Cfg {
   static constexpr int kA = 128 * 64 * 2;        // this CTA's 128 x 64 BF16 weight tile
   static constexpr int kB = (BN / 2) * 64 * 2;   // this CTA's half of the row tile
   static constexpr int kNumA = SWIGLU ? 2 : 1;
-  static constexpr int kStage = kA * kNumA + kB;
+  // 64-column K blocks per stage: two for the down projection, so that every
+  // stage carries eight MMAs like the gate/up stage (a stage's barrier round
+  // trip costs ~600 cycles, which four MMAs of a short row tile do not cover)
+  static constexpr int kKSub = SWIGLU ? 1 : 2;
+  static constexpr int kABytes = kA * kNumA * kKSub;
+  static constexpr int kStage = kABytes + kB * kKSub;
   static constexpr int kStages0 = (227 * 1024 - 2048) / kStage;
   static constexpr int kStages = kStages0 > 12 ? 12 : kStages0;
   static constexpr int kAccCols = kNumA * BN;
@@ -148,8 +153,8 @@ __global__ void __maxnreg__(kPairRegs)
         const int arow = un.mt * 256 + static_cast<int>(rank) * 128;
         const int brow = un.row0 + static_cast<int>(rank) * (n / 2);
         const CUtensorMap* bmap = &tmB.m[n / 32 - 1];  // box of n / 2 rows
-        const uint32_t tx = 2u * static_cast<uint32_t>(C::kA * C::kNumA + (n / 2) * 128);
-        for (int kb = 0; kb < args.k_blocks; ++kb, ++it) {
+        const uint32_t tx = 2u * static_cast<uint32_t>(C::kABytes + C::kKSub * (n / 2) * 128);
+        for (int ks = 0; ks < args.k_blocks / C::kKSub; ++ks, ++it) {
           const int s = it % C::kStages;
           const uint32_t ph = (it / C::kStages) & 1u;
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
@@ -158,9 +163,14 @@ __global__ void __maxnreg__(kPairRegs)
           }
           uint8_t* st = smem + s * C::kStage;
           if (rank == 0) mbar_arrive_expect_tx(&full[s], tx);
-          tma_load_3d_pair(st, &tmA0, &full[s], kb * 64, arow, un.g);
-          if (SWIGLU) tma_load_3d_pair(st + C::kA, &tmA1, &full[s], kb * 64, arow, un.g);
-          tma_load_2d_pair(st + C::kA * C::kNumA, bmap, &full[s], kb * 64, brow);
+#pragma unroll
+          for (int sub = 0; sub < C::kKSub; ++sub) {
+            const int kc = (ks * C::kKSub + sub) * 64;
+            uint8_t* a = st + sub * C::kNumA * C::kA;
+            tma_load_3d_pair(a, &tmA0, &full[s], kc, arow, un.g);
+            if (SWIGLU) tma_load_3d_pair(a + C::kA, &tmA1, &full[s], kc, arow, un.g);
+            tma_load_2d_pair(st + C::kABytes + sub * C::kB, bmap, &full[s], kc, brow);
+          }
           *issued = it + 1;
         }
       }
@@ -186,7 +196,7 @@ __global__ void __maxnreg__(kPairRegs)
         const uint32_t d0 = tmem_base + acc * C::kAccCols;
         const uint32_t n = static_cast<uint32_t>(((un.nvalid + 31) / 32) * 32);
         const uint32_t idesc = make_idesc(1u, n, 256);
-        for (int kb = 0; kb < args.k_blocks; ++kb, ++it) {
+        for (int ks = 0; ks < args.k_blocks / C::kKSub; ++ks, ++it) {
           const int s = it % C::kStages;
           const uint32_t ph = (it / C::kStages) & 1u;
           if (!mbar_wait(&full[s], ph, abort_flag)) {
@@ -195,14 +205,17 @@ __global__ void __maxnreg__(kPairRegs)
           }
           tc_fence_after();
           const uint32_t a0 = smem_u32(smem + s * C::kStage);
-          const uint64_t ad0 = sw128_kmajor_desc(a0);
-          const uint64_t ad1 = sw128_kmajor_desc(a0 + C::kA);
-          const uint64_t bd = sw128_kmajor_desc(a0 + C::kA * C::kNumA);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t accum = (kb | k) ? 1u : 0u;
-            mma_bf16_pair(d0, ad0 + 2 * k, bd + 2 * k, idesc, accum);
-            if (SWIGLU) mma_bf16_pair(d0 + BN, ad1 + 2 * k, bd + 2 * k, idesc, accum);
+          for (int sub = 0; sub < C::kKSub; ++sub) {
+            const uint64_t ad0 = sw128_kmajor_desc(a0 + sub * C::kNumA * C::kA);
+            const uint64_t ad1 = sw128_kmajor_desc(a0 + sub * C::kNumA * C::kA + C::kA);
+            const uint64_t bd = sw128_kmajor_desc(a0 + C::kABytes + sub * C::kB);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint32_t accum = (ks | sub | k) ? 1u : 0u;
+              mma_bf16_pair(d0, ad0 + 2 * k, bd + 2 * k, idesc, accum);
+              if (SWIGLU) mma_bf16_pair(d0 + BN, ad1 + 2 * k, bd + 2 * k, idesc, accum);
+            }
           }
           mma_commit_pair(&empty[s], 0x3);
           *consumed = it + 1;
