@@ -47,8 +47,9 @@ METRIC = "K2 MoE layer tokens/s; % of HBM (decode) / tensor-peak (prefill) roofl
 UNIT = "tokens/s"
 PHASES = ("router_logits", "router_topk", "route_scan", "dispatch", "gemm_gate_up",
           "gemm_down", "combine")
-KERNEL_SOURCES = {"gemm_gate_up": ["gemm_bf16.cu", "gemm_promoted.cu", "gemm_common.cuh", "sm100.cuh"],
-                  "gemm_down": ["gemm_bf16.cu", "gemm_promoted.cu", "gemm_common.cuh", "sm100.cuh"]}
+_GEMM_SOURCES = ["gemm_bf16.cu", "gemm_bf16_2sm.cu", "gemm_promoted.cu", "gemm_common.cuh",
+                 "sm100.cuh", "dispatch.cu"]
+KERNEL_SOURCES = {"gemm_gate_up": _GEMM_SOURCES, "gemm_down": _GEMM_SOURCES}
 
 
 # ----------------------------------------------------------------- workloads
