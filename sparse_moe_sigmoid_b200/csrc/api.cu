@@ -153,7 +153,7 @@ void free_all(moe_handle* h) {
   };
   f(h->w.router); f(h->w.router_cat); f(h->w.bias); f(h->w.gate); f(h->w.up); f(h->w.down);
   f(h->w.gate_s); f(h->w.up_s); f(h->w.down_s);
-  f(h->ws.logits_part); f(h->ws.ids); f(h->ws.wts); f(h->ws.counts); f(h->ws.word_prefix);
+  f(h->ws.logits_part); f(h->ws.ids); f(h->ws.wts); f(h->ws.sched); f(h->ws.word_prefix);
   f(h->ws.offsets); f(h->ws.unit_base); f(h->ws.pair_row); f(h->ws.row_token); f(h->ws.xp);
   f(h->ws.xs); f(h->ws.hbuf); f(h->ws.hs); f(h->ws.out); f(h->ws.status); f(h->ws.x_stage);
   f(h->ws.y_stage);
@@ -251,12 +251,13 @@ moe_status_t moe_create(const moe_config_t* cfg, int device, moe_handle_t** out)
   A(&h->ws.logits_part, part_rows * E * 4, "router partials");
   A(&h->ws.ids, Tm * dm.k * 4, "ids");
   A(&h->ws.wts, Tm * dm.k * 4, "weights");
-  h->ws.zero_bytes = E * 4 + E * W * 4;
+  h->ws.zero_bytes = 256 + E * 4 + E * W * 4;
   {
     void* z = nullptr;
     A(&z, h->ws.zero_bytes, "counts/bitmap");
-    h->ws.counts = static_cast<int32_t*>(z);
-    h->ws.bitmap = z ? reinterpret_cast<uint32_t*>(static_cast<char*>(z) + E * 4) : nullptr;
+    h->ws.sched = static_cast<int32_t*>(z);
+    h->ws.counts = z ? reinterpret_cast<int32_t*>(static_cast<char*>(z) + 256) : nullptr;
+    h->ws.bitmap = z ? reinterpret_cast<uint32_t*>(static_cast<char*>(z) + 256 + E * 4) : nullptr;
   }
   A(&h->ws.word_prefix, E * W * 4, "word prefix");
   A(&h->ws.offsets, (G + 1) * 4, "offsets");
@@ -437,7 +438,7 @@ moe_status_t moe_forward(moe_handle_t* h, const void* x, int64_t T, void* y,
   const int32_t* forced = opts ? opts->forced_topk_ids : nullptr;
 
   mark(0);
-  CUDA_TRY(h, cudaMemsetAsync(h->ws.counts, 0, h->ws.zero_bytes, s), "clear counts");
+  CUDA_TRY(h, cudaMemsetAsync(h->ws.sched, 0, h->ws.zero_bytes, s), "clear counts");
   const bool tensor_router = T >= smoe::kTensorRouterMinT;
   if (tensor_router) {
     CUDA_TRY(h, smoe::launch_router_gemm(h, x, Ti, s), "router GEMM launch");

@@ -25,6 +25,16 @@
 // gated accumulators fill TMEM (row tiles over 128, one buffer), the epilogue
 // computes h into packed BF16 registers, releases TMEM, and only then stores,
 // so the next unit's MMAs overlap the global stores.
+// Gate/up units are handed out dynamically (~55 long units per pair whose
+// cost varies with the row count): the even CTA's producer takes the next
+// unit index from a per-launch counter in global memory and publishes it
+// through a small ring in both CTAs' shared memory; the MMA thread, both
+// CTAs' epilogue warps and the odd CTA's producer read it from there and
+// release the slot. An index past the last unit ends every role's loop.
+// Down-projection units are short and many (~195 per pair, balanced by their
+// number): there every role walks the static sequence pair, pair + pairs, ...
+// (measured: the publication's cross-CTA latency at each unit start costs the
+// down GEMM more than dynamic balance gains).
 // Every wait is bounded as in gemm_bf16.cu. The only unbounded step is the
 // cluster barrier at entry and exit, which both CTAs always reach.
 #include <cuda_bf16.h>
@@ -40,6 +50,10 @@ using namespace sm100;
 
 constexpr int kPairBoxes = 8;     // activation box heights 16, 32, ..., 128 rows
 constexpr int kPairEpiWarps = 8;  // two per TMEM lane quarter
+constexpr int kUnitRing = 8;      // unit indices published ahead of the slowest reader
+// readers of each published unit index: the MMA thread, the epilogue warps of
+// both CTAs and the odd CTA's producer
+constexpr int kUnitReaders = 2 + 2 * kPairEpiWarps;
 constexpr int kPairThreads = 64 + 32 * kPairEpiWarps;
 // The register file is four 16K-register slices, one per SM sub-partition,
 // and warp w runs on slice w % 4: ten warps put three on a slice.
@@ -65,7 +79,7 @@ struct Pair2Cfg {
   static constexpr int kAccCols = kNumA * BN;
   static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
   static constexpr int kTmemCols = pow2_at_least(kAccBufs * kAccCols, 32);
-  static constexpr int kSmem = kStages * kStage + 1024 + 256;
+  static constexpr int kSmem = kStages * kStage + 1024 + 512;
   static_assert(BN % 32 == 0, "each CTA's half of the row tile is a multiple of 16 rows");
   static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(kTmemCols <= 512, "TMEM holds 512 columns");
@@ -100,7 +114,10 @@ __global__ void __maxnreg__(kPairRegs)
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* uq_full = drain + 1;           // [kUnitRing] a unit index was published
+  uint64_t* uq_empty = uq_full + kUnitRing;  // [kUnitRing] (even CTA) every reader has it
+  int32_t* uq = reinterpret_cast<int32_t*>(uq_empty + kUnitRing);  // [kUnitRing]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(uq + kUnitRing);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* consumed = tmem_slot + 2;
   volatile uint32_t* issued = tmem_slot + 3;
@@ -108,6 +125,7 @@ __global__ void __maxnreg__(kPairRegs)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs
+  const bool dynamic = args.sched != nullptr;
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
 
@@ -121,6 +139,10 @@ __global__ void __maxnreg__(kPairRegs)
       mbar_init(&tempty[a], 2 * kPairEpiWarps);  // the epilogue warps of both CTAs
     }
     mbar_init(drain, 1);
+    for (int j = 0; j < kUnitRing; ++j) {
+      mbar_init(&uq_full[j], 1);
+      mbar_init(&uq_empty[j], kUnitReaders);
+    }
     *abort_flag = 0;
     *consumed = 0;
     *issued = 0;
@@ -142,12 +164,57 @@ __global__ void __maxnreg__(kPairRegs)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total_units = total_units_of(args, BN);
+  // j-th unit index of this pair (every reader; false: a wait gave up)
+  auto read_unit = [&](uint32_t j, int* u) -> bool {
+    if (!dynamic) {
+      *u = pair + static_cast<int>(j) * npairs;
+      return true;
+    }
+    const int slot = static_cast<int>(j % kUnitRing);
+    const uint32_t ph = (j / kUnitRing) & 1u;
+    const bool ok = rank == 0 ? mbar_wait(&uq_full[slot], ph, abort_flag)
+                              : mbar_wait_cluster(&uq_full[slot], ph, abort_flag);
+    if (!ok) return false;
+    *u = uq[slot];
+    return true;
+  };
+  auto release_unit = [&](uint32_t j) {
+    if (!dynamic) return;
+    const int slot = static_cast<int>(j % kUnitRing);
+    if (rank == 0) mbar_arrive(&uq_empty[slot]);
+    else mbar_arrive_remote(&uq_empty[slot], 0);
+  };
 
   if (warp == 0) {
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      for (int u = pair; u < total_units && ok; u += npairs) {
+      // the even CTA takes unit indices one ahead, so the atomic's round trip
+      // overlaps the current unit's loads
+      int next_u = dynamic && rank == 0 ? atomicAdd(args.sched, 1) : 0;
+      for (uint32_t j = 0; ok; ++j) {
+        int u;
+        if (dynamic && rank == 0) {
+          // publish the next unit to both CTAs
+          const int slot = static_cast<int>(j % kUnitRing);
+          if (!mbar_wait_cluster(&uq_empty[slot], ((j / kUnitRing) & 1u) ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          u = next_u;
+          if (u < total_units) next_u = atomicAdd(args.sched, 1);
+          uq[slot] = u;
+          st_shared_remote_u32(&uq[slot], 1, static_cast<uint32_t>(u));
+          mbar_arrive(&uq_full[slot]);
+          mbar_arrive_remote(&uq_full[slot], 1);
+        } else {
+          if (!read_unit(j, &u)) {
+            ok = false;
+            break;
+          }
+          release_unit(j);
+        }
+        if (u >= total_units) break;
         const Unit un = decode_unit(u, args, BN);
         const int n = ((un.nvalid + 31) / 32) * 32;  // MMA N: halves of 16-row multiples
         const int arow = un.mt * 256 + static_cast<int>(rank) * 128;
@@ -183,8 +250,14 @@ __global__ void __maxnreg__(kPairRegs)
     if (lane == 0 && rank == 0) {
       uint32_t it = 0;
       bool ok = true;
-      int i = 0;
-      for (int u = pair; u < total_units && ok; u += npairs, ++i) {
+      for (uint32_t i = 0; ok; ++i) {
+        int u;
+        if (!read_unit(i, &u)) {
+          ok = false;
+          break;
+        }
+        release_unit(i);
+        if (u >= total_units) break;
         const Unit un = decode_unit(u, args, BN);
         const int acc = i % C::kAccBufs;
         const int use = i / C::kAccBufs;
@@ -233,8 +306,18 @@ __global__ void __maxnreg__(kPairRegs)
   } else {
     const int q = warp & 3;           // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;  // which alternate 16-column chunks
-    int i = 0;
-    for (int u = pair; u < total_units; u += npairs, ++i) {
+    for (uint32_t i = 0;; ++i) {
+      int u;
+      if (!read_unit(i, &u)) {
+        if (lane == 0) {
+          *abort_flag = 1;
+          atomicOr(args.status, MOE_DEVICE_WAIT_TIMEOUT);
+        }
+        break;
+      }
+      __syncwarp();
+      if (lane == 0) release_unit(i);
+      if (u >= total_units) break;
       const Unit un = decode_unit(u, args, BN);
       const int acc = i % C::kAccBufs;
       const int use = i / C::kAccBufs;
@@ -375,6 +458,7 @@ cudaError_t launch_gemm_bf16_pair(moe_handle* h, bool gated, const GemmPlan& p, 
   a.status = h->ws.status;
   a.b_k = gated ? dm.d : dm.f;
   a.m_valid = gated ? dm.f : dm.d;
+  a.sched = gated ? h->ws.sched : nullptr;  // dynamic units for gate/up only
   // activation maps with boxes of 16, 32, ..., 128 rows (each CTA's half of
   // a row tile of 32, 64, ..., 256)
   PairBoxMaps b;

@@ -41,6 +41,7 @@ struct GemmArgs {
   int m_valid;               // only output features < m_valid are stored
   int kpp;                   // promoted BF16 GEMM: stages accumulated in TMEM per promotion
   int stages;                // promoted GEMM: shared-memory ring depth
+  int32_t* sched;            // pair GEMM: unit counter, zero at launch (dynamic units); null: static
 };
 
 __device__ __forceinline__ int total_units_of(const GemmArgs& a, int BN) {

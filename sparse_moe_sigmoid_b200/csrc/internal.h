@@ -39,6 +39,7 @@ struct Workspace {
   float* logits_part = nullptr;   // [splits][T][E]
   int32_t* ids = nullptr;         // [T][k]
   float* wts = nullptr;           // [T][k]
+  int32_t* sched = nullptr;       // [64] unit counters of the pair GEMMs (zeroed per forward)
   int32_t* counts = nullptr;      // [E]            (zeroed per forward)
   uint32_t* bitmap = nullptr;     // [E][W] token bitmaps, W = ceil(Tmax/32) (zeroed per forward)
   int32_t* word_prefix = nullptr; // [E][W]
@@ -54,7 +55,7 @@ struct Workspace {
   uint32_t* status = nullptr;     // device status word
   void* x_stage = nullptr;        // [Tmax][d] BF16 staging for the host entry point
   void* y_stage = nullptr;        // [Tmax][d]
-  size_t zero_bytes = 0;          // bytes of the counts+bitmap region cleared per forward
+  size_t zero_bytes = 0;          // bytes of the sched+counts+bitmap region cleared per forward
 };
 
 struct Weights {

@@ -200,6 +200,39 @@ __device__ __forceinline__ void mbar_arrive_remote(uint64_t* bar, uint32_t cta) 
       : "memory");
 }
 
+// Store a 32-bit word at the same shared-memory offset in CTA `cta` of the cluster.
+__device__ __forceinline__ void st_shared_remote_u32(void* p, uint32_t cta, uint32_t v) {
+  asm volatile(
+      "{\n\t.reg .b32 ra;\n\t"
+      "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+      "st.shared::cluster.u32 [ra], %2;\n\t}" ::"r"(smem_u32(p)),
+      "r"(cta), "r"(v)
+      : "memory");
+}
+
+// mbar_wait with cluster-scope acquire: for phases completed by arrivals from
+// the other CTA of the pair that publish data in shared memory.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  volatile uint32_t* abort) {
+  const uint32_t addr = smem_u32(bar);
+  const uint64_t t0 = globaltimer();
+  for (uint32_t i = 0;; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(addr), "r"(parity), "r"(20u)
+        : "memory");
+    if (ok) return true;
+    if ((i & 31u) == 31u) {
+      if (abort != nullptr && *abort) return false;
+      if (globaltimer() - t0 > kTimeoutNs) return false;
+    }
+  }
+}
+
 // TMA load into this CTA's shared memory whose completion is counted on the
 // mbarrier at the same offset in the pair's even CTA (the address with the
 // CTA-rank bit cleared).
