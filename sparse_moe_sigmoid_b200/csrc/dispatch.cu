@@ -42,10 +42,10 @@ static int pick_bn(double want, const int* cands, int n) {
 #endif
 GemmPlan plan_gate_up(const Dims& dm, int64_t T) {
   static const int bf16_bn[] = {16, 32, 64, 96, 128, 160, 192, 224, 256};
-  static const int fp8_bn[] = {16, 32, 64};
+  static const int fp8_bn[] = {16, 32, 64, 96};
   const double want = SMOE_BN_FACTOR * static_cast<double>(T) * dm.k / dm.E;
   GemmPlan p;
-  p.bn = dm.fp8 ? pick_bn(want, fp8_bn, 3) : pick_bn(want, bf16_bn, 9);
+  p.bn = dm.fp8 ? pick_bn(want, fp8_bn, 4) : pick_bn(want, bf16_bn, 9);
   p.na = 2;
   p.pair = !dm.fp8 && pair_bn_supported(p.bn) && dm.f % 256 == 0;
   p.m_tiles = dm.f / (p.pair ? 256 : kBlock);
@@ -58,10 +58,10 @@ GemmPlan plan_gate_up(const Dims& dm, int64_t T) {
 // tiles of 128 and more) as one pair MMA over a CTA pair.
 GemmPlan plan_down(const Dims& dm, int64_t T) {
   static const int bf16_bn[] = {16, 32, 64, 96, 128, 160, 192, 224, 256};
-  static const int fp8_bn[] = {16, 32, 64, 128};
+  static const int fp8_bn[] = {16, 32, 64, 128, 192};
   const double want = SMOE_BN_FACTOR * static_cast<double>(T) * dm.k / dm.E;
   GemmPlan p;
-  p.bn = dm.fp8 ? pick_bn(want, fp8_bn, 4) : pick_bn(want, bf16_bn, 9);
+  p.bn = dm.fp8 ? pick_bn(want, fp8_bn, 5) : pick_bn(want, bf16_bn, 9);
   p.pair = !dm.fp8 && pair_bn_supported(p.bn) && dm.d % 256 == 0 && dm.f % 128 == 0;
   p.na = (!dm.fp8 && !p.pair && p.bn >= 64 && dm.d % 256 == 0) ? 2 : 1;
   p.m_tiles = dm.d / (p.pair ? 256 : kBlock * p.na);

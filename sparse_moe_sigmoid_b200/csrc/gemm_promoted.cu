@@ -59,6 +59,7 @@ template <int BN, bool GATED, bool FP8, int NPG>
 struct PromCfg {
   static constexpr int kThreads = 64 + 128 * NPG;
   static constexpr int kCols = BN / NPG;  // columns per promotion group
+  static constexpr int kBatch = NPG >= 3 ? 16 : kCols;  // TMEM columns per load batch
   static constexpr int kA = 128 * 128;    // 128 rows x 128 bytes of K
   static constexpr int kB = BN * 128;
   static constexpr int kKPerStage = FP8 ? 128 : 64;
@@ -292,32 +293,37 @@ __global__ void __maxnreg__(prom_regs<NPG>())
         const float sw0 = FP8 ? sw_s[pg] : 1.f;
         const float sw1 = (FP8 && GATED) ? sw_s[KB + pg] : 0.f;
         const float* sa = sa_s + pg * BN + c_begin;
-        // every load first, one wait, then the arithmetic: tcgen05.wait::ld
-        // waits for all outstanding loads, so a wait per chunk would pay the
-        // TMEM round trip once per chunk
-        uint32_t g[C::kCols], v[GATED ? C::kCols : 1];
+        // loads in batches of kBatch columns, one wait per batch, then the
+        // arithmetic: tcgen05.wait::ld waits for all outstanding loads, so a
+        // wait per 16-column chunk would pay the TMEM round trip once per
+        // chunk; with three groups the registers allow batches of 16 only
 #pragma unroll
-        for (int c = 0; c < C::kCols / 16; ++c) {
-          if (c_begin + c * 16 < un.nvalid) {
-            tmem_ld16(tq + pb * C::kPCols + c_begin + c * 16,
-                      *reinterpret_cast<uint32_t(*)[16]>(&g[c * 16]));
-            if (GATED)
-              tmem_ld16(tq + pb * C::kPCols + BN + c_begin + c * 16,
-                        *reinterpret_cast<uint32_t(*)[16]>(&v[c * 16]));
+        for (int b0 = 0; b0 < C::kCols; b0 += C::kBatch) {
+          uint32_t g[C::kBatch], v[GATED ? C::kBatch : 1];
+#pragma unroll
+          for (int c = 0; c < C::kBatch / 16; ++c) {
+            if (c_begin + b0 + c * 16 < un.nvalid) {
+              tmem_ld16(tq + pb * C::kPCols + c_begin + b0 + c * 16,
+                        *reinterpret_cast<uint32_t(*)[16]>(&g[c * 16]));
+              if (GATED)
+                tmem_ld16(tq + pb * C::kPCols + BN + c_begin + b0 + c * 16,
+                          *reinterpret_cast<uint32_t(*)[16]>(&v[c * 16]));
+            }
           }
-        }
-        tmem_ld_wait();
+          tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < C::kCols / 16; ++c) {
-          if (c_begin + c * 16 < un.nvalid) {
+          for (int c = 0; c < C::kBatch / 16; ++c) {
+            if (c_begin + b0 + c * 16 < un.nvalid) {
 #pragma unroll
-            for (int j = c * 16; j < c * 16 + 16; ++j) {
-              if (FP8) {
-                const float s = sa[j];
-                acc0[j] = fmaf(__uint_as_float(g[j]), sw0 * s, acc0[j]);
-                if (GATED) acc1[j] = fmaf(__uint_as_float(v[j]), sw1 * s, acc1[j]);
-              } else {
-                acc0[j] += __uint_as_float(g[j]);
+              for (int jj = c * 16; jj < c * 16 + 16; ++jj) {
+                const int j = b0 + jj;
+                if (FP8) {
+                  const float s = sa[j];
+                  acc0[j] = fmaf(__uint_as_float(g[jj]), sw0 * s, acc0[j]);
+                  if (GATED) acc1[j] = fmaf(__uint_as_float(v[jj]), sw1 * s, acc1[j]);
+                } else {
+                  acc0[j] += __uint_as_float(g[jj]);
+                }
               }
             }
           }
@@ -449,6 +455,7 @@ cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaSt
       case 16: return launch_one<16, true, true, 1>(h, g, u, b, a, s);
       case 32: return launch_one<32, true, true, 1>(h, g, u, b, a, s);
       case 64: return launch_one<64, true, true, 2>(h, g, u, b, a, s);
+      case 96: return launch_one<96, true, true, 3>(h, g, u, b, a, s);
       default: return cudaErrorInvalidValue;
     }
   }
@@ -464,6 +471,7 @@ cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaSt
     case 32: return launch_one<32, false, true, 1>(h, w, w, b, a, s);
     case 64: return launch_one<64, false, true, 1>(h, w, w, b, a, s);
     case 128: return launch_one<128, false, true, 2>(h, w, w, b, a, s);
+    case 192: return launch_one<192, false, true, 3>(h, w, w, b, a, s);
     default: return cudaErrorInvalidValue;
   }
 }

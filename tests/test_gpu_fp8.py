@@ -120,13 +120,17 @@ def test_fp8_on_grid_matches_bf16(smoe):
 
 @pytest.fixture(scope="module")
 def k2fp8(smoe):
-    layer = gu.make_layer(synth.K2, 1024, "fp8")
-    h = gu.create_handle(smoe, layer, max_tokens=1024)
+    layer = gu.make_layer(synth.K2, 8192, "fp8")
+    h = gu.create_handle(smoe, layer, max_tokens=8192)
     yield layer, h
     smoe.moe_destroy(h)
 
 
-@pytest.mark.parametrize("T,n_sample", [(1, 1), (16, 4), (128, 4), (1024, 4)])
+# T = 4096 and 8192 reach the tallest FP8 row tiles (96 rows gate/up with three
+# promotion warpgroups; 128 and 192 rows down); routing is checked for every
+# token, outputs on a seeded sample
+@pytest.mark.parametrize("T,n_sample", [(1, 1), (16, 4), (128, 4), (1024, 4), (4096, 6),
+                                        (8192, 6)])
 def test_k2_fp8(smoe, k2fp8, T, n_sample):
     layer, h = k2fp8
     x = layer.x[:T].contiguous()
