@@ -226,7 +226,9 @@ moe_status_t moe_create(const moe_config_t* cfg, int device, moe_handle_t** out)
   size_t part_rows = 0;
   for (int64_t T = 64;; T += 64) {
     const int64_t Tc = T < dm.Tmax ? T : dm.Tmax;
-    const size_t rows = static_cast<size_t>(smoe::router_splits(dm, Tc, h->num_sms)) * Tc;
+    const int sp = Tc >= smoe::kTensorRouterMinT ? smoe::kTensorRouterSplits
+                                                 : smoe::router_splits(dm, Tc, h->num_sms);
+    const size_t rows = static_cast<size_t>(sp) * Tc;
     if (rows > part_rows) part_rows = rows;
     if (Tc == dm.Tmax) break;
   }
@@ -446,7 +448,7 @@ moe_status_t moe_forward(moe_handle_t* h, const void* x, int64_t T, void* y,
     CUDA_TRY(h, smoe::launch_router_logits(h, x, Ti, splits, s), "router logits launch");
   }
   mark(1);
-  CUDA_TRY(h, smoe::launch_router_topk(h, Ti, tensor_router ? 1 : splits, forced, s,
+  CUDA_TRY(h, smoe::launch_router_topk(h, Ti, tensor_router ? smoe::kTensorRouterSplits : splits, forced, s,
                                        opts ? opts->topk_ids_out : nullptr,
                                        opts ? opts->topk_weights_out : nullptr,
                                        opts ? opts->router_logits_out : nullptr),

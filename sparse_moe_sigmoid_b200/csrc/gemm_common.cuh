@@ -20,6 +20,7 @@ struct Unit {
   int mt;      // 128-feature tile
   int row0;    // first row of the row tile
   int nvalid;  // rows of the tile that belong to g (1..BN)
+  int split;   // K slice (single-group mode with ksplit > 1), else 0
 };
 
 struct GemmArgs {
@@ -42,15 +43,25 @@ struct GemmArgs {
   int kpp;                   // promoted BF16 GEMM: stages accumulated in TMEM per promotion
   int stages;                // promoted GEMM: shared-memory ring depth
   int32_t* sched;            // pair GEMM: unit counter, zero at launch (dynamic units); null: static
+  int ksplit;                // single-group mode: K slices per tile (0 or 1: none); slice s
+                             // covers k-blocks [s, s+1) * k_blocks / ksplit and writes its
+                             // partial result at out + s * split_stride elements
+  size_t split_stride;
 };
 
 __device__ __forceinline__ int total_units_of(const GemmArgs& a, int BN) {
-  return a.unit_base ? __ldg(a.unit_base + a.G) : a.m_tiles * ((a.single_rows + BN - 1) / BN);
+  return a.unit_base ? __ldg(a.unit_base + a.G)
+                     : a.m_tiles * ((a.single_rows + BN - 1) / BN) * (a.ksplit > 1 ? a.ksplit : 1);
 }
 
 __device__ __forceinline__ Unit decode_unit(int u, const GemmArgs& a, int BN) {
   Unit un;
+  un.split = 0;
   if (a.unit_base == nullptr) {
+    if (a.ksplit > 1) {  // the K slices of one tile are adjacent units
+      un.split = u % a.ksplit;
+      u /= a.ksplit;
+    }
     const int nt = (a.single_rows + BN - 1) / BN;
     un.g = 0;
     un.mt = u / nt;

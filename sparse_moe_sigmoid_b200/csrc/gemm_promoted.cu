@@ -107,7 +107,7 @@ __global__ void __maxnreg__(prom_regs<NPG>())
                                  const __grid_constant__ CUtensorMap tmA1,
                                  const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
   using C = PromCfg<BN, GATED, FP8, NPG>;
-  const int KB = args.k_blocks;
+  const int KB = args.k_blocks / (args.ksplit > 1 ? args.ksplit : 1);  // k-blocks per unit
   const int S = args.stages;  // ring depth, set at launch (<= kPromMaxStages)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -178,7 +178,7 @@ __global__ void __maxnreg__(prom_regs<NPG>())
           }
           uint8_t* st = smem + s * C::kStage;
           mbar_arrive_expect_tx(&full[s], C::kStage);
-          const int kc = kb * C::kKPerStage;
+          const int kc = (un.split * KB + kb) * C::kKPerStage;
           tma_load_3d(st, &tmA0, &full[s], kc, un.mt * 128, un.g);
           if (GATED) tma_load_3d(st + C::kA, &tmA1, &full[s], kc, un.mt * 128, un.g);
           tma_load_2d(st + C::kA * C::kNumA, &tmB, &full[s], kc % args.b_k, un.row0);
@@ -368,7 +368,7 @@ __global__ void __maxnreg__(prom_regs<NPG>())
           }
         }
       } else {
-        float* out = static_cast<float*>(args.out);
+        float* out = static_cast<float*>(args.out) + un.split * args.split_stride;
         if (feat < args.m_valid) {
 #pragma unroll
           for (int j = 0; j < C::kCols; ++j)
@@ -481,7 +481,9 @@ cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaSt
 // significand bits cover fp32's 24), concatenated along K. x (BF16) times
 // each part is an exact product; partial sums over 128 K are promoted into
 // fp32 registers (see the file comment). One group of T rows; B's K index
-// wraps onto x's d columns.
+// wraps onto x's d columns. Each part is its own K slice (kTensorRouterSplits
+// partial logits, added by the top-k kernel), which also triples the units so
+// that the grid runs close to whole waves.
 cudaError_t launch_router_gemm(moe_handle* h, const void* x, int T, cudaStream_t s) {
   const Dims& dm = h->dims;
   constexpr int BN = 128;
@@ -502,6 +504,8 @@ cudaError_t launch_router_gemm(moe_handle* h, const void* x, int T, cudaStream_t
   a.single_rows = T;
   a.m_tiles = (dm.E + 127) / 128;
   a.k_blocks = 3 * dm.d / 64;
+  a.ksplit = kTensorRouterSplits;
+  a.split_stride = static_cast<size_t>(T) * dm.E;
   a.kpp = 2;
   a.bn = BN;
   a.b_k = dm.d;

@@ -104,6 +104,7 @@ cudaError_t launch_router_split(moe_handle* h, cudaStream_t s);
 // gemm_promoted.cu: the router's logits on the tensor cores (T >= kTensorRouterMinT)
 cudaError_t launch_router_gemm(moe_handle* h, const void* x, int T, cudaStream_t s);
 constexpr int kTensorRouterMinT = 512;
+constexpr int kTensorRouterSplits = 3;  // one K slice per BF16 part of the router weight
 cudaError_t launch_router_raw(const void* x, const float* router_weight, const float* bias, int T,
                               int d, int E, int k, float scale, int norm, int splits, float* part,
                               int32_t* counts, uint32_t* bitmap, int W, uint32_t* status,
