@@ -11,8 +11,8 @@
 // K = 32 per instruction, 4 per 128-column block) into an fp32 partial in
 // TMEM; the scales differ per block, so each block's partial is promoted
 // separately: four promotion warps read it (tcgen05.ld), multiply by
-// s_w * s_x[row] and add into fp32 registers. The partial lives in two TMEM
-// buffers used in turn, so the MMAs of block kb+1 run while block kb is
+// s_w * s_x[row] and add into fp32 registers. The partial rotates through up
+// to four TMEM buffers, so the MMAs of the next blocks run while block kb is
 // promoted. (The hardware's own block scaling takes power-of-two ue8m0
 // scales per 32 columns; the K2 scales are arbitrary fp32 per 128, so it does
 // not apply.)
@@ -67,12 +67,19 @@ struct PromCfg {
   static constexpr int kStage = kA * kNumA + kB;
   static constexpr int kAmaxBytes = GATED ? 4 * BN * 4 : 0;
   static constexpr int kPCols = GATED ? 2 * BN : BN;  // one partial buffer
-  static constexpr int kTmemCols = pow2_at_least(2 * kPCols, 32);
+  // partial buffers in TMEM: as many as fit (up to 4), so that the MMAs can
+  // run several blocks ahead of the promotion (a hand-over costs an MMA
+  // completion plus two mbarrier wake-ups, several hundred cycles)
+  static constexpr int kPBufs = 512 / pow2_at_least(kPCols, 32) >= 4   ? 4
+                                : 512 / pow2_at_least(kPCols, 32) >= 2 ? 2
+                                                                       : 1;
+  static constexpr int kTmemCols = pow2_at_least(kPBufs * kPCols, 32);
   static constexpr int kBarrierBytes = 512;
   static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(kCols % 16 == 0, "columns per group in 16-column loads");
   static_assert((GATED ? 2 : 1) * kCols <= 64, "one promotion's loads must fit in registers");
   static_assert(kTmemCols <= 512, "TMEM holds 512 columns");
+  static_assert(kPBufs >= 2, "the promotion needs two partial buffers at least");
   static_assert(FP8 || !GATED, "the BF16 promoted GEMM is plain");
   // scale staging of FP8: activation scales [KB][BN] and weight scales [2][KB]
   static constexpr int scale_bytes(int kb) { return FP8 ? (kb * BN + 2 * kb) * 4 : 0; }
@@ -119,8 +126,8 @@ __global__ void __maxnreg__(prom_regs<NPG>())
       (reinterpret_cast<uintptr_t>(amax_s + (GATED ? 4 * BN : 0)) + 7) & ~uintptr_t(7));
   uint64_t* empty = full + kPromMaxStages;
   uint64_t* pfull = empty + kPromMaxStages;
-  uint64_t* pempty = pfull + 2;
-  uint64_t* drain = pempty + 2;
+  uint64_t* pempty = pfull + 4;
+  uint64_t* drain = pempty + 4;
   uint64_t* grp = drain + 1;  // the promotion threads' own barrier (bounded waits)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(grp + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
@@ -136,7 +143,7 @@ __global__ void __maxnreg__(prom_regs<NPG>())
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < C::kPBufs; ++a) {
       mbar_init(&pfull[a], 1);
       mbar_init(&pempty[a], 4 * NPG);
     }
@@ -202,9 +209,10 @@ __global__ void __maxnreg__(prom_regs<NPG>())
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1u;
-          const int pb = pit & 1;
+          const int pb = pit % C::kPBufs;
           const int sub = kb % KPP;
-          if ((sub == 0 && !mbar_wait(&pempty[pb], ((pit >> 1) & 1u) ^ 1u, abort_flag)) ||
+          if ((sub == 0 &&
+               !mbar_wait(&pempty[pb], ((pit / C::kPBufs) & 1u) ^ 1u, abort_flag)) ||
               !mbar_wait(&full[s], ph, abort_flag)) {
             ok = false;
             break;
@@ -284,8 +292,8 @@ __global__ void __maxnreg__(prom_regs<NPG>())
       }
       const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
       for (int pg = 0; pg < NP; ++pg, ++pit) {
-        const int pb = pit & 1;
-        if (!mbar_wait(&pfull[pb], (pit >> 1) & 1u, abort_flag)) {
+        const int pb = pit % C::kPBufs;
+        if (!mbar_wait(&pfull[pb], (pit / C::kPBufs) & 1u, abort_flag)) {
           ok = false;
           break;
         }
