@@ -17,7 +17,7 @@ constexpr int kMaxTopK = 32;
 constexpr int kMaxExperts = 512;
 constexpr int kRouterTile = 64;   // router tile: 64 tokens x 64 experts
 constexpr int kRouterKTile = 32;
-constexpr int kRouterMaxSplits = 16;
+constexpr int kRouterMaxSplits = 32;
 
 // Sizes derived from the config, fixed per handle.
 struct Dims {

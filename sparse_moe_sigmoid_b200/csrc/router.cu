@@ -67,42 +67,42 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const __nv_bfloat16*
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 
+  // global loads of K tile k0 + kRouterKTile are issued before tile k0 is
+  // multiplied (register double buffering: the loop is latency-bound at the
+  // small T this kernel serves)
+  const bool t_ok = t0 + lr < T, e_ok = e0 + lr < E;
+  const __nv_bfloat16* xrow = x + (size_t)(t0 + lr) * d + lc;
+  const float* wrow = W + (size_t)(e0 + lr) * d + lc;
+  uint4 xr = make_uint4(0u, 0u, 0u, 0u);
+  float4 wa = make_float4(0.f, 0.f, 0.f, 0.f), wb = wa;
+  if (kbeg < kend) {
+    if (t_ok) xr = *reinterpret_cast<const uint4*>(xrow + kbeg);
+    if (e_ok) {
+      wa = *reinterpret_cast<const float4*>(wrow + kbeg);
+      wb = *reinterpret_cast<const float4*>(wrow + kbeg + 4);
+    }
+  }
   for (int k0 = kbeg; k0 < kend; k0 += kRouterKTile) {
     {
-      const int t = t0 + lr;
-      float v[8];
-      if (t < T) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(x + (size_t)t * d + k0 + lc);
-        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&xr);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 f2 = __bfloat1622float2(p[i]);
-          v[2 * i] = f2.x;
-          v[2 * i + 1] = f2.y;
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = 0.f;
+      for (int i = 0; i < 4; ++i) {
+        const float2 f2 = __bfloat1622float2(p[i]);
+        Xs[lc + 2 * i][lr] = f2.x;
+        Xs[lc + 2 * i + 1][lr] = f2.y;
       }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) Xs[lc + i][lr] = v[i];
-    }
-    {
-      const int e = e0 + lr;
-      float v[8];
-      if (e < E) {
-        const float4 a = *reinterpret_cast<const float4*>(W + (size_t)e * d + k0 + lc);
-        const float4 b = *reinterpret_cast<const float4*>(W + (size_t)e * d + k0 + lc + 4);
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = 0.f;
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) Ws[lc + i][lr] = v[i];
+      Ws[lc + 0][lr] = wa.x; Ws[lc + 1][lr] = wa.y; Ws[lc + 2][lr] = wa.z; Ws[lc + 3][lr] = wa.w;
+      Ws[lc + 4][lr] = wb.x; Ws[lc + 5][lr] = wb.y; Ws[lc + 6][lr] = wb.z; Ws[lc + 7][lr] = wb.w;
     }
     __syncthreads();
+    const int kn = k0 + kRouterKTile;
+    if (kn < kend) {
+      if (t_ok) xr = *reinterpret_cast<const uint4*>(xrow + kn);
+      if (e_ok) {
+        wa = *reinterpret_cast<const float4*>(wrow + kn);
+        wb = *reinterpret_cast<const float4*>(wrow + kn + 4);
+      }
+    }
 #pragma unroll
     for (int kk = 0; kk < kRouterKTile; ++kk) {
       const float4 a = *reinterpret_cast<const float4*>(&Xs[kk][ty * 4]);
@@ -141,13 +141,25 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
   if (t >= T) return;
   const unsigned full = 0xffffffffu;
 
-  float key[kPerLane], sc[kPerLane];
+  float key[kPerLane], sc[kPerLane], lg[kPerLane];
+#pragma unroll
+  for (int i = 0; i < kPerLane; ++i) lg[i] = 0.f;
+  // slices in order (a deterministic sum); the loads of a slice's experts are
+  // independent, so they are issued together, four slices at a time
+#pragma unroll 4
+  for (int s = 0; s < splits; ++s) {
+    const float* ps = part + ((size_t)s * T + t) * E;
+    float v[kPerLane];
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i) v[i] = lane + 32 * i < E ? __ldg(ps + lane + 32 * i) : 0.f;
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i) lg[i] += v[i];
+  }
 #pragma unroll
   for (int i = 0; i < kPerLane; ++i) {
     const int e = lane + 32 * i;
     if (e < E) {
-      float l = 0.f;
-      for (int s = 0; s < splits; ++s) l += part[((size_t)s * T + t) * E + e];
+      const float l = lg[i];
       if (logits_out) logits_out[(size_t)t * E + e] = l;
       const float p = 1.f / (1.f + expf(-l));
       sc[i] = p;
