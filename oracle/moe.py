@@ -18,7 +18,7 @@ What the layer computes, and where the pages fix it:
     activation scheme -- the same page's config.json quantization_config
     excerpt and its "one scale per 128 x 128 block" evidence note.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent (the library follows the same ones):
   R1 router weight fp32, logits accumulated exactly (float64 here).
   R2 noaux_tc: key = sigmoid score + e_score_correction_bias; the bias only
      chooses experts, the weights use the unbiased scores.
