@@ -334,12 +334,17 @@ def run_native(args, wl):
     yh = torch.empty_like(xh).pin_memory()
     for _ in range(2):
         smoe.moe_forward_host(h, xh, yh)
+        smoe.moe_forward_host_async(h, xh, yh)
+    smoe.moe_host_wait(h)
     n_e2e = max(3, min(args.steps, 50))
     barrier(dev)
     torch.cuda.synchronize()
     e0.record(stream)
     for _ in range(n_e2e):
-        smoe.moe_forward_host(h, xh, yh)  # copies in, forward, copy out, synchronise
+        # every step: upload x from pinned memory, forward, download y; the
+        # library overlaps each step's copies with its neighbours' forwards
+        smoe.moe_forward_host_async(h, xh, yh)
+    smoe.moe_host_wait(h)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / n_e2e
@@ -393,7 +398,9 @@ def run_native(args, wl):
         "cpu_baseline": cpu,
         "e2e": {"value": tokens_all / (e2e_ms / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 2),
-                "ms_per_step": e2e_ms, "api": "moe_forward_host (pinned host x and y)"},
+                "ms_per_step": e2e_ms,
+                "api": "moe_forward_host_async + moe_host_wait (pinned host x and y; uploads and "
+                       "downloads overlap neighbouring forwards)"},
         "gpu_launches": int(launches),
         "clocks": clk,
     }

@@ -155,12 +155,29 @@ moe_status_t moe_load_weights(moe_handle_t* h, const moe_weights_t* w, void* str
 moe_status_t moe_forward(moe_handle_t* h, const void* x, int64_t T, void* y,
                          const moe_forward_opts_t* opts, void* stream);
 
-/* The same forward from and to host memory: copies x_host (BF16 [T, d]) to
- * the device, runs moe_forward, copies y back into y_host, all on `stream`,
- * then synchronises the stream. Page-locked host buffers give the fastest
- * copies; pageable ones work. */
+/* The same forward from and to host memory, returning once y_host holds the
+ * result: moe_forward_host_async followed by moe_host_wait. x_host and y_host
+ * are BF16 [T, d]. Page-locked host buffers give the fastest copies;
+ * pageable ones work (their copies are then synchronous). */
 moe_status_t moe_forward_host(moe_handle_t* h, const void* x_host, int64_t T, void* y_host,
                               const moe_forward_opts_t* opts, void* stream);
+
+/* Pipelined host-memory forward. Enqueues, without waiting: the copy of x_host
+ * into one of two device staging buffers (used in turn) on the handle's
+ * upload stream; the forward on `stream`; the copy of the result into y_host
+ * on the handle's download stream. So the upload of the next call overlaps
+ * this call's forward, and this call's download overlaps the next forward.
+ * A staging buffer is reused only after the forward (x) and the download (y)
+ * of the call two earlier are done. The caller must not change x_host, nor
+ * read y_host, until moe_host_wait returns; calls may use the same buffers
+ * (each download then overwrites the previous one in order). Argument checks
+ * and errors as moe_forward; one handle, one host thread at a time. */
+moe_status_t moe_forward_host_async(moe_handle_t* h, const void* x_host, int64_t T, void* y_host,
+                                    const moe_forward_opts_t* opts, void* stream);
+
+/* Block until every upload, forward and download enqueued by
+ * moe_forward_host_async on this handle has finished. */
+moe_status_t moe_host_wait(moe_handle_t* h);
 
 /* Synchronise the handle's device, return the device status word in
  * *flags (MOE_DEVICE_* bits) and clear it. */

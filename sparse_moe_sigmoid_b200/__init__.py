@@ -76,6 +76,9 @@ _sig = {
                          ctypes.POINTER(moe_forward_opts_t), ctypes.c_void_p]),
     "moe_forward_host": (_S, [_H, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                               ctypes.POINTER(moe_forward_opts_t), ctypes.c_void_p]),
+    "moe_forward_host_async": (_S, [_H, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                    ctypes.POINTER(moe_forward_opts_t), ctypes.c_void_p]),
+    "moe_host_wait": (_S, [_H]),
     "moe_get_device_status": (_S, [_H, ctypes.POINTER(ctypes.c_uint32)]),
     "moe_profile_enable": (_S, [_H, ctypes.c_int32]),
     "moe_profile_read": (_S, [_H, ctypes.POINTER(ctypes.c_float), ctypes.c_int32,
@@ -190,6 +193,20 @@ def moe_forward_host(h, x_host, y_host, T: Optional[int] = None, flags: int = 0,
     st = _lib.moe_forward_host(h, _ptr(x_host), T, _ptr(y_host),
                                _opts(None, None, None, None, flags), _stream(stream))
     _check(st, "moe_forward_host", h)
+
+
+def moe_forward_host_async(h, x_host, y_host, T: Optional[int] = None, flags: int = 0,
+                           stream=None):
+    """Pipelined host-memory forward (returns at once); keep x_host unchanged and
+    y_host unread, and both alive, until moe_host_wait(h) returns."""
+    T = x_host.shape[0] if T is None else T
+    st = _lib.moe_forward_host_async(h, _ptr(x_host), T, _ptr(y_host),
+                                     _opts(None, None, None, None, flags), _stream(stream))
+    _check(st, "moe_forward_host_async", h)
+
+
+def moe_host_wait(h):
+    _check(_lib.moe_host_wait(h), "moe_host_wait", h)
 
 
 def moe_get_device_status(h) -> int:

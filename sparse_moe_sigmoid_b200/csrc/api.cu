@@ -155,8 +155,18 @@ void free_all(moe_handle* h) {
   f(h->w.gate_s); f(h->w.up_s); f(h->w.down_s);
   f(h->ws.logits_part); f(h->ws.ids); f(h->ws.wts); f(h->ws.sched); f(h->ws.word_prefix);
   f(h->ws.offsets); f(h->ws.unit_base); f(h->ws.pair_row); f(h->ws.row_token); f(h->ws.xp);
-  f(h->ws.xs); f(h->ws.hbuf); f(h->ws.hs); f(h->ws.out); f(h->ws.status); f(h->ws.x_stage);
-  f(h->ws.y_stage);
+  f(h->ws.xs); f(h->ws.hbuf); f(h->ws.hs); f(h->ws.out); f(h->ws.status);
+  for (int b = 0; b < 2; ++b) {
+    f(h->ws.x_stage[b]);
+    f(h->ws.y_stage[b]);
+    if (h->ev_x[b]) cudaEventDestroy(h->ev_x[b]);
+    if (h->ev_fwd[b]) cudaEventDestroy(h->ev_fwd[b]);
+    if (h->ev_y[b]) cudaEventDestroy(h->ev_y[b]);
+    h->ev_x[b] = h->ev_fwd[b] = h->ev_y[b] = nullptr;
+  }
+  if (h->up) cudaStreamDestroy(h->up);
+  if (h->down) cudaStreamDestroy(h->down);
+  h->up = h->down = nullptr;
   for (cudaEvent_t e : h->prof_events) cudaEventDestroy(e);
   h->prof_events.clear();
 }
@@ -274,8 +284,19 @@ moe_status_t moe_create(const moe_config_t* cfg, int device, moe_handle_t** out)
   }
   A(&h->ws.out, Rm * d * 4, "expert outputs");
   A(&h->ws.status, 4, "status");
-  A(&h->ws.x_stage, Tm * d * 2, "x staging");
-  A(&h->ws.y_stage, Tm * d * 2, "y staging");
+  for (int b = 0; b < 2; ++b) {
+    A(&h->ws.x_stage[b], Tm * d * 2, "x staging");
+    A(&h->ws.y_stage[b], Tm * d * 2, "y staging");
+  }
+  if (rc == MOE_OK) {
+    bool ok = cudaStreamCreateWithFlags(&h->up, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&h->down, cudaStreamNonBlocking) == cudaSuccess;
+    for (int b = 0; b < 2 && ok; ++b)
+      ok = cudaEventCreateWithFlags(&h->ev_x[b], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&h->ev_fwd[b], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&h->ev_y[b], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) rc = MOE_ERR_CUDA;
+  }
   if (rc != MOE_OK) {
     free_all(h);
     delete h;
@@ -489,8 +510,8 @@ moe_status_t moe_forward(moe_handle_t* h, const void* x, int64_t T, void* y,
   return MOE_OK;
 }
 
-moe_status_t moe_forward_host(moe_handle_t* h, const void* x_host, int64_t T, void* y_host,
-                              const moe_forward_opts_t* opts, void* stream) {
+moe_status_t moe_forward_host_async(moe_handle_t* h, const void* x_host, int64_t T, void* y_host,
+                                    const moe_forward_opts_t* opts, void* stream) {
   if (h == nullptr) return MOE_ERR_INVALID_ARG;
   if (T < 0 || T > h->dims.Tmax) return fail(h, MOE_ERR_INVALID_ARG, "T outside [0, max_tokens]");
   if (T == 0) return MOE_OK;
@@ -501,12 +522,42 @@ moe_status_t moe_forward_host(moe_handle_t* h, const void* x_host, int64_t T, vo
   if (!guard.ok) return fail(h, MOE_ERR_CUDA, "cudaSetDevice failed");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t nbytes = static_cast<size_t>(T) * h->dims.d * 2;
-  CUDA_TRY(h, cudaMemcpyAsync(h->ws.x_stage, x_host, nbytes, cudaMemcpyHostToDevice, s), "x copy");
-  moe_status_t st = moe_forward(h, h->ws.x_stage, T, h->ws.y_stage, opts, stream);
+  const int b = static_cast<int>(h->host_calls & 1);
+  // upload into staging b once the forward that read it (two calls ago) is done
+  CUDA_TRY(h, cudaStreamWaitEvent(h->up, h->ev_fwd[b], 0), "upload wait");
+  CUDA_TRY(h, cudaMemcpyAsync(h->ws.x_stage[b], x_host, nbytes, cudaMemcpyHostToDevice, h->up),
+           "x copy");
+  CUDA_TRY(h, cudaEventRecord(h->ev_x[b], h->up), "upload event");
+  // the forward on the caller's stream: after the upload, and once y staging
+  // b has been downloaded (two calls ago)
+  CUDA_TRY(h, cudaStreamWaitEvent(s, h->ev_x[b], 0), "forward wait");
+  CUDA_TRY(h, cudaStreamWaitEvent(s, h->ev_y[b], 0), "forward wait");
+  moe_status_t st = moe_forward(h, h->ws.x_stage[b], T, h->ws.y_stage[b], opts, stream);
   if (st != MOE_OK) return st;
-  CUDA_TRY(h, cudaMemcpyAsync(y_host, h->ws.y_stage, nbytes, cudaMemcpyDeviceToHost, s), "y copy");
-  CUDA_TRY(h, cudaStreamSynchronize(s), "stream sync");
+  CUDA_TRY(h, cudaEventRecord(h->ev_fwd[b], s), "forward event");
+  // download after the forward
+  CUDA_TRY(h, cudaStreamWaitEvent(h->down, h->ev_fwd[b], 0), "download wait");
+  CUDA_TRY(h, cudaMemcpyAsync(y_host, h->ws.y_stage[b], nbytes, cudaMemcpyDeviceToHost, h->down),
+           "y copy");
+  CUDA_TRY(h, cudaEventRecord(h->ev_y[b], h->down), "download event");
+  ++h->host_calls;
   return MOE_OK;
+}
+
+moe_status_t moe_host_wait(moe_handle_t* h) {
+  if (h == nullptr) return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return fail(h, MOE_ERR_CUDA, "cudaSetDevice failed");
+  CUDA_TRY(h, cudaStreamSynchronize(h->up), "upload sync");
+  CUDA_TRY(h, cudaStreamSynchronize(h->down), "download sync");  // follows every forward
+  return MOE_OK;
+}
+
+moe_status_t moe_forward_host(moe_handle_t* h, const void* x_host, int64_t T, void* y_host,
+                              const moe_forward_opts_t* opts, void* stream) {
+  moe_status_t st = moe_forward_host_async(h, x_host, T, y_host, opts, stream);
+  if (st != MOE_OK || T == 0) return st;
+  return moe_host_wait(h);
 }
 
 moe_status_t moe_get_device_status(moe_handle_t* h, uint32_t* flags) {

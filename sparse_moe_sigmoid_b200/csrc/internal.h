@@ -53,8 +53,8 @@ struct Workspace {
   float* hs = nullptr;            // [Rmax][f/128] FP8 scales of h
   float* out = nullptr;           // [Rmax][d] fp32 per-row expert outputs
   uint32_t* status = nullptr;     // device status word
-  void* x_stage = nullptr;        // [Tmax][d] BF16 staging for the host entry point
-  void* y_stage = nullptr;        // [Tmax][d]
+  void* x_stage[2] = {};          // [Tmax][d] BF16 staging of the host entry points, used in turn
+  void* y_stage[2] = {};          // [Tmax][d]
   size_t zero_bytes = 0;          // bytes of the sched+counts+bitmap region cleared per forward
 };
 
@@ -90,6 +90,11 @@ struct moe_handle {
   // per-phase profiling
   std::vector<cudaEvent_t> prof_events;
   int prof_cap = 0, prof_next = 0;
+  // host-memory entry points: upload and download streams, and per staging
+  // buffer b the events "x uploaded", "forward done", "y downloaded"
+  cudaStream_t up = nullptr, down = nullptr;
+  cudaEvent_t ev_x[2] = {}, ev_fwd[2] = {}, ev_y[2] = {};
+  uint64_t host_calls = 0;
 };
 
 namespace smoe {

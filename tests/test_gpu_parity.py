@@ -160,6 +160,31 @@ def test_host_entry_point_matches_device(smoe, tiny):
     assert torch.equal(yh, y_dev.cpu())
 
 
+def test_host_pipeline_matches_device(smoe, tiny):
+    """Pipelined host calls (two staging buffers used in turn, uploads and
+    downloads on their own streams): each call's result equals moe_forward's
+    on the same input, for calls 3 and 4 that reuse calls 1 and 2's staging
+    buffers, and for repeated calls on one pair of host buffers."""
+    layer, h = tiny
+    T = layer.x.shape[0]
+    xs = [layer.x, layer.x.flip(0).contiguous(), (layer.x * 0.5).contiguous(),
+          layer.x.roll(7, 0).contiguous()]
+    want = [gu.run(smoe, h, layer, x)[0].cpu() for x in xs]
+    xh = [x.cpu().pin_memory() for x in xs]
+    yh = [torch.empty_like(x).pin_memory() for x in xh]
+    for i in range(4):
+        smoe.moe_forward_host_async(h, xh[i], yh[i])
+    smoe.moe_host_wait(h)
+    for i in range(4):
+        assert torch.equal(yh[i], want[i]), i
+    # the same host buffers every call (each download overwrites the last)
+    yone = torch.empty_like(xh[0]).pin_memory()
+    for i in range(3):
+        smoe.moe_forward_host_async(h, xh[1], yone, T=T)
+    smoe.moe_host_wait(h)
+    assert torch.equal(yone, want[1])
+
+
 def test_profile_phases(smoe, tiny):
     layer, h = tiny
     smoe.moe_profile_enable(h, 3)
