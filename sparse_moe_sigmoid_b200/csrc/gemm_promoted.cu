@@ -55,18 +55,22 @@ constexpr int kPromSmemBudget = 227 * 1024 - 2048;
 
 // FP8: e4m3 operands, 128 K per stage, block scales applied at promotion.
 // Otherwise BF16 operands, 64 K per stage, no scales.
-template <int BN, bool GATED, bool FP8, int NPG>
+// DUAL (FP8 down projection, short row tiles): two consecutive 128-feature
+// weight tiles per unit, loaded, multiplied and promoted like gate and up,
+// both stored as fp32 outputs, so that a stage carries two weight tiles.
+template <int BN, bool GATED, bool FP8, int NPG, bool DUAL = false>
 struct PromCfg {
+  static constexpr bool kTwoA = GATED || DUAL;
   static constexpr int kThreads = 64 + 128 * NPG;
   static constexpr int kCols = BN / NPG;  // columns per promotion group
   static constexpr int kBatch = NPG >= 3 ? 16 : kCols;  // TMEM columns per load batch
   static constexpr int kA = 128 * 128;    // 128 rows x 128 bytes of K
   static constexpr int kB = BN * 128;
   static constexpr int kKPerStage = FP8 ? 128 : 64;
-  static constexpr int kNumA = GATED ? 2 : 1;
+  static constexpr int kNumA = kTwoA ? 2 : 1;
   static constexpr int kStage = kA * kNumA + kB;
   static constexpr int kAmaxBytes = GATED ? 4 * BN * 4 : 0;
-  static constexpr int kPCols = GATED ? 2 * BN : BN;  // one partial buffer
+  static constexpr int kPCols = kTwoA ? 2 * BN : BN;  // one partial buffer
   // partial buffers in TMEM: as many as fit (up to 4), so that the MMAs can
   // run several blocks ahead of the promotion (a hand-over costs an MMA
   // completion plus two mbarrier wake-ups, several hundred cycles)
@@ -77,7 +81,8 @@ struct PromCfg {
   static constexpr int kBarrierBytes = 512;
   static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(kCols % 16 == 0, "columns per group in 16-column loads");
-  static_assert((GATED ? 2 : 1) * kCols <= 64, "one promotion's loads must fit in registers");
+  static_assert((kTwoA ? 2 : 1) * kCols <= 64, "one promotion's loads must fit in registers");
+  static_assert(!(GATED && DUAL) && (FP8 || !DUAL), "DUAL is the plain FP8 mode");
   static_assert(kTmemCols <= 512, "TMEM holds 512 columns");
   static_assert(kPBufs >= 2, "the promotion needs two partial buffers at least");
   static_assert(FP8 || !GATED, "the BF16 promoted GEMM is plain");
@@ -108,12 +113,12 @@ constexpr int prom_regs() {
   return prom_max_regs<64 + 128 * NPG>();
 }
 
-template <int BN, bool GATED, bool FP8, int NPG>
+template <int BN, bool GATED, bool FP8, int NPG, bool DUAL>
 __global__ void __maxnreg__(prom_regs<NPG>())
     grouped_gemm_promoted_kernel(const __grid_constant__ CUtensorMap tmA0,
                                  const __grid_constant__ CUtensorMap tmA1,
                                  const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
-  using C = PromCfg<BN, GATED, FP8, NPG>;
+  using C = PromCfg<BN, GATED, FP8, NPG, DUAL>;
   const int KB = args.k_blocks / (args.ksplit > 1 ? args.ksplit : 1);  // k-blocks per unit
   const int S = args.stages;  // ring depth, set at launch (<= kPromMaxStages)
   extern __shared__ uint8_t smem_raw[];
@@ -157,7 +162,7 @@ __global__ void __maxnreg__(prom_regs<NPG>())
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA0);
-    if (GATED) tma_prefetch_desc(&tmA1);
+    if (C::kTwoA) tma_prefetch_desc(&tmA1);
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
@@ -186,8 +191,9 @@ __global__ void __maxnreg__(prom_regs<NPG>())
           uint8_t* st = smem + s * C::kStage;
           mbar_arrive_expect_tx(&full[s], C::kStage);
           const int kc = (un.split * KB + kb) * C::kKPerStage;
-          tma_load_3d(st, &tmA0, &full[s], kc, un.mt * 128, un.g);
-          if (GATED) tma_load_3d(st + C::kA, &tmA1, &full[s], kc, un.mt * 128, un.g);
+          const int arow = DUAL ? un.mt * 256 : un.mt * 128;
+          tma_load_3d(st, &tmA0, &full[s], kc, arow, un.g);
+          if (C::kTwoA) tma_load_3d(st + C::kA, &tmA1, &full[s], kc, arow + (DUAL ? 128 : 0), un.g);
           tma_load_2d(st + C::kA * C::kNumA, &tmB, &full[s], kc % args.b_k, un.row0);
           *issued = it + 1;
         }
@@ -228,7 +234,7 @@ __global__ void __maxnreg__(prom_regs<NPG>())
             const uint32_t accum = (k | sub) ? 1u : 0u;  // each promotion's partial starts fresh
             if (FP8) {
               mma_fp8(d0, ad0 + 2 * k, bd + 2 * k, idesc, accum);
-              if (GATED) mma_fp8(d0 + BN, ad1 + 2 * k, bd + 2 * k, idesc, accum);
+              if (C::kTwoA) mma_fp8(d0 + BN, ad1 + 2 * k, bd + 2 * k, idesc, accum);
             } else {
               mma_bf16(d0, ad0 + 2 * k, bd + 2 * k, idesc, accum);
             }
@@ -273,10 +279,14 @@ __global__ void __maxnreg__(prom_regs<NPG>())
           const int kb = i / BN, j = i - kb * BN;
           sa_s[i] = j < un.nvalid ? __ldg(args.act_scale + (size_t)(un.row0 + j) * KB + kb) : 0.f;
         }
-        const size_t wrow = ((size_t)un.g * args.m_tiles + un.mt) * KB;
+        // weight block scales [G][rows / 128][KB]: the tile's row of blocks
+        // (DUAL: the two consecutive rows of its two tiles)
+        const size_t wrow = DUAL ? ((size_t)un.g * 2 * args.m_tiles + 2 * un.mt) * KB
+                                 : ((size_t)un.g * args.m_tiles + un.mt) * KB;
         for (int i = ptid; i < KB; i += 128 * NPG) {
           sw_s[i] = __ldg(args.w_scale0 + wrow + i);
           if (GATED) sw_s[KB + i] = __ldg(args.w_scale1 + wrow + i);
+          if (DUAL) sw_s[KB + i] = __ldg(args.w_scale0 + wrow + KB + i);
         }
         if (!group_sync()) {
           ok = false;
@@ -284,11 +294,11 @@ __global__ void __maxnreg__(prom_regs<NPG>())
         }
       }
 
-      float acc0[C::kCols], acc1[GATED ? C::kCols : 1];
+      float acc0[C::kCols], acc1[C::kTwoA ? C::kCols : 1];
 #pragma unroll
       for (int j = 0; j < C::kCols; ++j) {
         acc0[j] = 0.f;
-        if (GATED) acc1[j] = 0.f;
+        if (C::kTwoA) acc1[j] = 0.f;
       }
       const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
       for (int pg = 0; pg < NP; ++pg, ++pit) {
@@ -299,7 +309,7 @@ __global__ void __maxnreg__(prom_regs<NPG>())
         }
         tc_fence_after();
         const float sw0 = FP8 ? sw_s[pg] : 1.f;
-        const float sw1 = (FP8 && GATED) ? sw_s[KB + pg] : 0.f;
+        const float sw1 = (FP8 && C::kTwoA) ? sw_s[KB + pg] : 0.f;
         const float* sa = sa_s + pg * BN + c_begin;
         // loads in batches of kBatch columns, one wait per batch, then the
         // arithmetic: tcgen05.wait::ld waits for all outstanding loads, so a
@@ -307,13 +317,13 @@ __global__ void __maxnreg__(prom_regs<NPG>())
         // chunk; with three groups the registers allow batches of 16 only
 #pragma unroll
         for (int b0 = 0; b0 < C::kCols; b0 += C::kBatch) {
-          uint32_t g[C::kBatch], v[GATED ? C::kBatch : 1];
+          uint32_t g[C::kBatch], v[C::kTwoA ? C::kBatch : 1];
 #pragma unroll
           for (int c = 0; c < C::kBatch / 16; ++c) {
             if (c_begin + b0 + c * 16 < un.nvalid) {
               tmem_ld16(tq + pb * C::kPCols + c_begin + b0 + c * 16,
                         *reinterpret_cast<uint32_t(*)[16]>(&g[c * 16]));
-              if (GATED)
+              if (C::kTwoA)
                 tmem_ld16(tq + pb * C::kPCols + BN + c_begin + b0 + c * 16,
                           *reinterpret_cast<uint32_t(*)[16]>(&v[c * 16]));
             }
@@ -328,7 +338,7 @@ __global__ void __maxnreg__(prom_regs<NPG>())
                 if (FP8) {
                   const float s = sa[j];
                   acc0[j] = fmaf(__uint_as_float(g[jj]), sw0 * s, acc0[j]);
-                  if (GATED) acc1[j] = fmaf(__uint_as_float(v[jj]), sw1 * s, acc1[j]);
+                  if (C::kTwoA) acc1[j] = fmaf(__uint_as_float(v[jj]), sw1 * s, acc1[j]);
                 } else {
                   acc0[j] += __uint_as_float(g[jj]);
                 }
@@ -377,11 +387,18 @@ __global__ void __maxnreg__(prom_regs<NPG>())
         }
       } else {
         float* out = static_cast<float*>(args.out) + un.split * args.split_stride;
-        if (feat < args.m_valid) {
+        const int f0 = DUAL ? un.mt * 256 + q * 32 + lane : feat;
+        if (f0 < args.m_valid) {
 #pragma unroll
           for (int j = 0; j < C::kCols; ++j)
             if (c_begin + j < un.nvalid)
-              out[static_cast<size_t>(un.row0 + c_begin + j) * args.ld + feat] = acc0[j];
+              out[static_cast<size_t>(un.row0 + c_begin + j) * args.ld + f0] = acc0[j];
+        }
+        if (DUAL && f0 + 128 < args.m_valid) {
+#pragma unroll
+          for (int j = 0; j < C::kCols; ++j)
+            if (c_begin + j < un.nvalid)
+              out[static_cast<size_t>(un.row0 + c_begin + j) * args.ld + f0 + 128] = acc1[j];
         }
       }
     }
@@ -403,13 +420,14 @@ __global__ void __maxnreg__(prom_regs<NPG>())
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
-template <int BN, bool GATED, bool FP8, int NPG>
+template <int BN, bool GATED, bool FP8, int NPG, bool DUAL = false>
 static cudaError_t launch_one(moe_handle* h, const CUtensorMap& a0, const CUtensorMap& a1,
                               const CUtensorMap& b, GemmArgs args, cudaStream_t s) {
-  using C = PromCfg<BN, GATED, FP8, NPG>;
+  using C = PromCfg<BN, GATED, FP8, NPG, DUAL>;
+  auto kern = grouped_gemm_promoted_kernel<BN, GATED, FP8, NPG, DUAL>;
   static bool configured[64] = {};
   if (h->device < 64 && !configured[h->device]) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_promoted_kernel<BN, GATED, FP8, NPG>,
+    cudaError_t e = cudaFuncSetAttribute(kern,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kPromSmemBudget + 1024);
     if (e != cudaSuccess) return e;
@@ -418,13 +436,13 @@ static cudaError_t launch_one(moe_handle* h, const CUtensorMap& a0, const CUtens
   args.stages = C::stages(args.k_blocks);
   if (args.stages < 2) return cudaErrorInvalidValue;
   const int smem = C::smem(args.k_blocks);
-  grouped_gemm_promoted_kernel<BN, GATED, FP8, NPG><<<h->num_sms, C::kThreads, smem, s>>>(
+  kern<<<h->num_sms, C::kThreads, smem, s>>>(
       a0, a1, b, args);
   h->launches++;
   const cudaError_t e = cudaGetLastError();
   if (e == cudaErrorLaunchOutOfResources) {
     cudaFuncAttributes fa{};
-    cudaFuncGetAttributes(&fa, grouped_gemm_promoted_kernel<BN, GATED, FP8, NPG>);
+    cudaFuncGetAttributes(&fa, kern);
     char buf[256];
     snprintf(buf, sizeof buf,
              "promoted GEMM BN=%d: %d threads x %d registers, %zu B local, max threads %d, "
@@ -447,7 +465,7 @@ cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaSt
   a.bn = p.bn;
   a.status = h->ws.status;
   a.b_k = gated ? dm.d : dm.f;
-  a.m_valid = p.m_tiles * 128;
+  a.m_valid = gated ? dm.f : dm.d;
   const int bi = bn_index(p.bn);
   if (bi < 0) return cudaErrorInvalidValue;
   if (gated) {
@@ -474,6 +492,14 @@ cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaSt
   a.act_scale = h->ws.hs;
   const CUtensorMap& b = h->tm_h[bi];
   const CUtensorMap& w = h->tm_down;
+  if (p.na == 2) {
+    switch (p.bn) {
+      case 16: return launch_one<16, false, true, 1, true>(h, w, w, b, a, s);
+      case 32: return launch_one<32, false, true, 1, true>(h, w, w, b, a, s);
+      case 64: return launch_one<64, false, true, 2, true>(h, w, w, b, a, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (p.bn) {
     case 16: return launch_one<16, false, true, 1>(h, w, w, b, a, s);
     case 32: return launch_one<32, false, true, 1>(h, w, w, b, a, s);
