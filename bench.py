@@ -11,6 +11,8 @@ Workloads (--config):
   decode      K2 layer, T = 64 tokens, BF16 experts (default)
   prefill     K2 layer, T = 8192 tokens, BF16 experts
   fp8-T<n>    K2 layer, T = n tokens, FP8 e4m3 experts with 128x128 scales
+  dense-T<n>  K2's dense FFN layer (its first layer: one SwiGLU MLP of
+              intermediate 18432, no router), T = n tokens, BF16 (dense-fp8-T<n>: FP8)
 
 N > 1 runs one independent replica per GPU (data parallel over token
 batches; the layer has no exchange step at one GPU per replica), so the
@@ -58,6 +60,13 @@ def workload(name: str):
         return dict(T=64, fmt="bf16", desc="K2 MoE layer decode step, T=64 tokens, BF16 experts")
     if name == "prefill":
         return dict(T=8192, fmt="bf16", desc="K2 MoE layer prefill, T=8192 tokens, BF16 experts")
+    if name.startswith("dense-"):
+        fmt = "fp8" if name.startswith("dense-fp8-T") else "bf16"
+        T = int(name.split("T")[-1])
+        shape = synth.LayerShape(n_routed_experts=0, num_experts_per_tok=0, n_shared_experts=9)
+        return dict(T=T, fmt=fmt, shape=shape,
+                    desc=f"K2 dense FFN layer (intermediate 18432 = 9 x 2048, no router), "
+                         f"T={T} tokens, {fmt.upper()} weights")
     if name.startswith("fp8-T"):
         T = int(name[5:])
         return dict(T=T, fmt="fp8", desc=f"K2 MoE layer, T={T} tokens, FP8 e4m3 experts "
@@ -181,6 +190,11 @@ class OracleSample:
         self.Wg = Wg_cpu.numpy().astype(np.float64)
         self.b = b_cpu.numpy().astype(np.float64)
         self.tok = np.sort(rng.choice(T, size=min(n_tok, T), replace=False))
+        self.shared = fetch_expert(-1) if shape.n_shared_experts > 0 else None
+        self.dense = shape.n_routed_experts == 0
+        if self.dense:  # no router: the shared MLP alone
+            self.rows = self.tok
+            return
         rows = np.union1d(self.tok, rng.choice(T, size=self.route_rows, replace=False))
         self.rows = rows
         r = orc.route(self.x[rows], self.Wg, self.b, shape.num_experts_per_tok,
@@ -188,11 +202,13 @@ class OracleSample:
         pos = np.searchsorted(rows, self.tok)
         need = sorted(set(int(e) for e in r.ids[pos].ravel()))
         self.cache = {e: fetch_expert(e) for e in need}
-        self.shared = fetch_expert(-1) if shape.n_shared_experts > 0 else None
         self.pos = pos
 
     def run_once(self) -> int:
         s, orc = self.shape, self.orc
+        if self.dense:
+            orc.dense_ffn(self.x[self.tok], self.shared, self.fmt)
+            return len(self.tok)
         r = orc.route(self.x[self.rows], self.Wg, self.b, s.num_experts_per_tok,
                       s.routed_scaling_factor, s.norm_topk_prob)
         orc.experts_combine(self.x[self.rows], r.ids, r.weights, lambda e: self.cache[e],
@@ -201,6 +217,9 @@ class OracleSample:
         return len(self.tok)
 
     def describe(self):
+        if self.dense:
+            return (f"{len(self.tok)} of {self.T} tokens through the dense FFN, weights "
+                    "preloaded on the host")
         return (f"{len(self.tok)} of {self.T} tokens through the experts (routing for "
                 f"{len(self.rows)} tokens), weights preloaded on the host")
 
@@ -270,6 +289,7 @@ def run_native(args, wl):
     ew = synth.make_experts(shape, device=dev, fmt=fmt)
     cfg = smoe.moe_config_init_k2(
         max_tokens=T, n_routed_experts=shape.n_routed_experts,
+        num_experts_per_tok=shape.num_experts_per_tok, n_shared_experts=shape.n_shared_experts,
         weight_format=smoe.MOE_WEIGHT_BF16 if fmt == "bf16" else smoe.MOE_WEIGHT_FP8_E4M3_BLOCK)
     h = smoe.moe_create(cfg, local)
     smoe.moe_load_weights(h, Wg, b, ew.gate, ew.up, ew.down, ew.shared_gate, ew.shared_up,
@@ -387,7 +407,7 @@ def run_native(args, wl):
         "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) weights, random init)",
         "config": {"workload": wl["desc"], "tokens": T, "global_batch": T * ws,
                    "hidden_size": shape.hidden_size, "n_routed_experts": shape.n_routed_experts,
-                   "top_k": shape.num_experts_per_tok, "moe_intermediate_size":
+                   "top_k": shape.num_experts_per_tok, "n_shared_experts": shape.n_shared_experts, "moe_intermediate_size":
                        shape.moe_intermediate_size, "parallelism": f"replicas x{ws}",
                    "distinct_experts_hit": alg["U"],
                    "l2": "no flush: the expert weights streamed each step exceed the 126 MB L2"},
@@ -437,7 +457,7 @@ def run_reference(args, wl):
         "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) weights, random init)",
         "config": {"workload": wl["desc"], "tokens": T, "global_batch": T * ws,
                    "hidden_size": shape.hidden_size, "n_routed_experts": shape.n_routed_experts,
-                   "top_k": shape.num_experts_per_tok,
+                   "top_k": shape.num_experts_per_tok, "n_shared_experts": shape.n_shared_experts,
                    "moe_intermediate_size": shape.moe_intermediate_size,
                    "parallelism": "host cores, rank 0 only"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",

@@ -77,9 +77,15 @@ typedef enum { MOE_ACTIVATION_DYNAMIC = 0 } moe_activation_scheme_t;
 typedef struct {
   int32_t hidden_size;            /* d: 7168 for K2; multiple of 128, <= 16384 */
   int32_t moe_intermediate_size;  /* f: 2048 for K2; multiple of 128, <= 8192 */
-  int32_t n_routed_experts;       /* E: 384 for K2; 1..512 */
-  int32_t num_experts_per_tok;    /* k: 8 for K2; 1..min(E, 32) */
-  int32_t n_shared_experts;       /* 1 for K2; 0..8 (intermediate f * n_shared) */
+  int32_t n_routed_experts;       /* E: 384 for K2; 1..512, or 0 (below) */
+  int32_t num_experts_per_tok;    /* k: 8 for K2; 1..min(E, 32); 0 when E = 0 */
+  int32_t n_shared_experts;       /* 1 for K2; 0..16 (intermediate f * n_shared) */
+  /* E = 0, k = 0, n_shared_experts >= 1: no routed experts and no router; the
+   * layer is the shared SwiGLU MLP alone, a dense FFN of intermediate
+   * f * n_shared_experts. K2's first layer ("Kimi K2 Base" config:
+   * first_k_dense_replace 1, intermediate_size 18432) is f = 2048,
+   * n_shared_experts = 9. The router and routed-expert weights are then
+   * ignored (may be NULL). */
   int32_t n_group;                /* must be 1 (K2) */
   int32_t topk_group;             /* must be 1 (K2) */
   int32_t norm_topk_prob;         /* 1 (K2): normalise the k scores; 0: do not */

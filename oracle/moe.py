@@ -223,6 +223,22 @@ def experts_combine(x: np.ndarray, ids: np.ndarray, weights: np.ndarray,
     return y
 
 
+def dense_ffn(x: np.ndarray, mats: Dict[str, np.ndarray], fmt: str = "bf16") -> np.ndarray:
+    """The model's dense FFN layer, its first layer ("Behind Kimi-K2's Config"
+    §2.3: first_k_dense = 1; "Kimi K2 Base" raw config fields:
+    first_k_dense_replace 1, intermediate_size 18432, hidden_act silu):
+    y = down(silu(gate x) * up x) over intermediate_size columns, no router.
+    The pages print this formula for the experts ("Kimi K2 · Down
+    projection"); the dense layer is read as the same MLP. mats holds
+    gate [i, d], up [i, d], down [d, i] (BF16 values, or FP8 codes with their
+    *_scale block scales, dequantised and with x and h quantised as for the
+    experts)."""
+    x = np.asarray(x, np.float64)
+    m = _as_f64_expert(mats, fmt)
+    ffn = swiglu_expert if fmt == "bf16" else swiglu_expert_fp8
+    return ffn(x, m["gate"], m["up"], m["down"])
+
+
 def forward(x, router_weight, bias, get_expert: ExpertFn, get_shared, k: int,
             routed_scaling_factor: float = 2.827, norm_topk_prob: bool = True,
             fmt: str = "bf16", n_shared_experts: int = 1,

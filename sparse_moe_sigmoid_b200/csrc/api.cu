@@ -112,9 +112,16 @@ moe_status_t validate(const moe_config_t* c, std::string* why) {
     *why = m;
     return MOE_ERR_UNSUPPORTED;
   };
-  if (c->hidden_size <= 0 || c->moe_intermediate_size <= 0 || c->n_routed_experts <= 0 ||
-      c->num_experts_per_tok <= 0 || c->n_shared_experts < 0 || c->max_tokens <= 0)
+  if (c->hidden_size <= 0 || c->moe_intermediate_size <= 0 || c->n_routed_experts < 0 ||
+      c->num_experts_per_tok < 0 || c->n_shared_experts < 0 || c->max_tokens <= 0)
     return bad("sizes must be positive (n_shared_experts >= 0)");
+  if (c->n_routed_experts == 0) {
+    // no routed experts: the layer is its shared MLP alone (a dense FFN)
+    if (c->num_experts_per_tok != 0 || c->n_shared_experts < 1)
+      return bad("without routed experts: num_experts_per_tok 0 and n_shared_experts >= 1");
+  } else if (c->num_experts_per_tok <= 0) {
+    return bad("num_experts_per_tok must be positive");
+  }
   if (c->num_experts_per_tok > c->n_routed_experts)
     return bad("num_experts_per_tok > n_routed_experts");
   if (c->hidden_size % 128 || c->moe_intermediate_size % 128)
@@ -123,7 +130,7 @@ moe_status_t validate(const moe_config_t* c, std::string* why) {
     return unsup("hidden_size <= 16384 and moe_intermediate_size <= 8192");
   if (c->n_routed_experts > smoe::kMaxExperts) return unsup("n_routed_experts > 512");
   if (c->num_experts_per_tok > smoe::kMaxTopK) return unsup("num_experts_per_tok > 32");
-  if (c->n_shared_experts > 8) return unsup("n_shared_experts > 8");
+  if (c->n_shared_experts > 16) return unsup("n_shared_experts > 16");
   if (c->n_group != 1 || c->topk_group != 1)
     return unsup("group-limited routing (n_group/topk_group != 1) is not implemented");
   if (c->scoring_func != MOE_SCORING_SIGMOID) return unsup("scoring_func must be sigmoid");
@@ -234,7 +241,7 @@ moe_status_t moe_create(const moe_config_t* cfg, int device, moe_handle_t** out)
 
   // the router's split-K partial buffer: largest splits(T) * T over T <= Tmax
   size_t part_rows = 0;
-  for (int64_t T = 64;; T += 64) {
+  for (int64_t T = 64; dm.E > 0; T += 64) {
     const int64_t Tc = T < dm.Tmax ? T : dm.Tmax;
     const int sp = Tc >= smoe::kTensorRouterMinT ? smoe::kTensorRouterSplits
                                                  : smoe::router_splits(dm, Tc, h->num_sms);
@@ -330,8 +337,8 @@ moe_status_t moe_create(const moe_config_t* cfg, int device, moe_handle_t** out)
     uint64_t dims[3] = {3 * d, E, 1};
     uint64_t str[2] = {3 * d * 2, E * 3 * d * 2};
     uint32_t box[3] = {64, 128, 1};
-    ok = ok && smoe::make_tmap(&h->tm_router, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, h->w.router_cat,
-                               dims, str, box, &why);
+    ok = ok && (E == 0 || smoe::make_tmap(&h->tm_router, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                                          h->w.router_cat, dims, str, box, &why));
   }
   for (int i = 0; i < 16 && ok; ++i) {
     const uint32_t bn = 16u * (i + 1);
@@ -355,12 +362,12 @@ moe_status_t moe_create(const moe_config_t* cfg, int device, moe_handle_t** out)
 moe_status_t moe_load_weights(moe_handle_t* h, const moe_weights_t* w, void* stream) {
   if (h == nullptr || w == nullptr) return MOE_ERR_INVALID_ARG;
   const Dims& dm = h->dims;
-  if (!w->router_weight || !w->e_score_correction_bias || !w->gate_proj || !w->up_proj ||
-      !w->down_proj)
+  if (dm.E > 0 && (!w->router_weight || !w->e_score_correction_bias || !w->gate_proj ||
+                   !w->up_proj || !w->down_proj))
     return fail(h, MOE_ERR_INVALID_ARG, "router, bias and routed expert weights are required");
   if (dm.ns > 0 && (!w->shared_gate_proj || !w->shared_up_proj || !w->shared_down_proj))
     return fail(h, MOE_ERR_INVALID_ARG, "shared expert weights are required");
-  if (dm.fp8 && (!w->gate_scale || !w->up_scale || !w->down_scale ||
+  if (dm.fp8 && ((dm.E > 0 && (!w->gate_scale || !w->up_scale || !w->down_scale)) ||
                  (dm.ns > 0 && (!w->shared_gate_scale || !w->shared_up_scale ||
                                 !w->shared_down_scale))))
     return fail(h, MOE_ERR_INVALID_ARG, "FP8 weights need every block-scale tensor");
@@ -375,17 +382,20 @@ moe_status_t moe_load_weights(moe_handle_t* h, const moe_weights_t* w, void* str
   };
   auto bytes_to = [](void* p, size_t off) { return static_cast<char*>(p) + off; };
 
-  CUDA_TRY(h, cudaMemcpyAsync(h->w.router, w->router_weight, E * d * 4, K, s), "router copy");
-  CUDA_TRY(h, cudaMemcpyAsync(h->w.bias, w->e_score_correction_bias, E * 4, K, s), "bias copy");
-  CUDA_TRY(h, smoe::launch_router_split(h, s), "router split launch");
-  CUDA_TRY(h, cudaMemcpyAsync(h->w.gate, w->gate_proj, E * f * d * wb, K, s), "gate copy");
-  CUDA_TRY(h, cudaMemcpyAsync(h->w.up, w->up_proj, E * f * d * wb, K, s), "up copy");
-  CUDA_TRY(h, cudaMemcpyAsync(h->w.down, w->down_proj, E * d * f * wb, K, s), "down copy");
   const size_t nb_f = f / 128, nb_d = d / 128, nb_fs = fs / 128;
-  if (dm.fp8) {
-    CUDA_TRY(h, cudaMemcpyAsync(h->w.gate_s, w->gate_scale, E * nb_f * nb_d * 4, K, s), "scales");
-    CUDA_TRY(h, cudaMemcpyAsync(h->w.up_s, w->up_scale, E * nb_f * nb_d * 4, K, s), "scales");
-    CUDA_TRY(h, cudaMemcpyAsync(h->w.down_s, w->down_scale, E * nb_d * nb_f * 4, K, s), "scales");
+  if (E > 0) {  // router and routed experts (none in a dense FFN layer)
+    CUDA_TRY(h, cudaMemcpyAsync(h->w.router, w->router_weight, E * d * 4, K, s), "router copy");
+    CUDA_TRY(h, cudaMemcpyAsync(h->w.bias, w->e_score_correction_bias, E * 4, K, s), "bias copy");
+    CUDA_TRY(h, smoe::launch_router_split(h, s), "router split launch");
+    CUDA_TRY(h, cudaMemcpyAsync(h->w.gate, w->gate_proj, E * f * d * wb, K, s), "gate copy");
+    CUDA_TRY(h, cudaMemcpyAsync(h->w.up, w->up_proj, E * f * d * wb, K, s), "up copy");
+    CUDA_TRY(h, cudaMemcpyAsync(h->w.down, w->down_proj, E * d * f * wb, K, s), "down copy");
+    if (dm.fp8) {
+      CUDA_TRY(h, cudaMemcpyAsync(h->w.gate_s, w->gate_scale, E * nb_f * nb_d * 4, K, s), "scales");
+      CUDA_TRY(h, cudaMemcpyAsync(h->w.up_s, w->up_scale, E * nb_f * nb_d * 4, K, s), "scales");
+      CUDA_TRY(h, cudaMemcpyAsync(h->w.down_s, w->down_scale, E * nb_d * nb_f * 4, K, s),
+               "scales");
+    }
   }
   // shared expert of intermediate fs = ns * f -> ns groups of f: gate/up take
   // row slices, down takes column slices (a pitched copy)
@@ -457,23 +467,30 @@ moe_status_t moe_forward(moe_handle_t* h, const void* x, int64_t T, void* y,
 
   const GemmPlan p1 = smoe::plan_gate_up(dm, T);
   const GemmPlan p2 = smoe::plan_down(dm, T);
-  const int splits = smoe::router_splits(dm, T, h->num_sms);
+  const int splits = dm.E > 0 ? smoe::router_splits(dm, T, h->num_sms) : 0;
   const int32_t* forced = opts ? opts->forced_topk_ids : nullptr;
 
   mark(0);
   CUDA_TRY(h, cudaMemsetAsync(h->ws.sched, 0, h->ws.zero_bytes, s), "clear counts");
+  // without routed experts (a dense FFN layer) there is nothing to route: the
+  // router phases are empty and the shared groups take every token
   const bool tensor_router = T >= smoe::kTensorRouterMinT;
-  if (tensor_router) {
-    CUDA_TRY(h, smoe::launch_router_gemm(h, x, Ti, s), "router GEMM launch");
-  } else {
-    CUDA_TRY(h, smoe::launch_router_logits(h, x, Ti, splits, s), "router logits launch");
+  if (dm.E > 0) {
+    if (tensor_router) {
+      CUDA_TRY(h, smoe::launch_router_gemm(h, x, Ti, s), "router GEMM launch");
+    } else {
+      CUDA_TRY(h, smoe::launch_router_logits(h, x, Ti, splits, s), "router logits launch");
+    }
   }
   mark(1);
-  CUDA_TRY(h, smoe::launch_router_topk(h, Ti, tensor_router ? smoe::kTensorRouterSplits : splits, forced, s,
-                                       opts ? opts->topk_ids_out : nullptr,
-                                       opts ? opts->topk_weights_out : nullptr,
-                                       opts ? opts->router_logits_out : nullptr),
-           "router top-k launch");
+  if (dm.E > 0) {
+    CUDA_TRY(h,
+             smoe::launch_router_topk(h, Ti, tensor_router ? smoe::kTensorRouterSplits : splits,
+                                      forced, s, opts ? opts->topk_ids_out : nullptr,
+                                      opts ? opts->topk_weights_out : nullptr,
+                                      opts ? opts->router_logits_out : nullptr),
+             "router top-k launch");
+  }
   mark(2);
   CUDA_TRY(h, smoe::launch_route_scan(h, Ti, p1, p2, s), "route scan launch");
   mark(3);

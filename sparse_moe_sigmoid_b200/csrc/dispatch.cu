@@ -40,10 +40,16 @@ static int pick_bn(double want, const int* cands, int n) {
 #ifndef SMOE_BN_FACTOR
 #define SMOE_BN_FACTOR 1.5  // tuning constant
 #endif
+// mean rows per routed expert (T k / E); every token's row in each shared
+// group when there are no routed experts
+static double rows_per_group(const Dims& dm, int64_t T) {
+  return dm.E > 0 ? static_cast<double>(T) * dm.k / dm.E : static_cast<double>(T);
+}
+
 GemmPlan plan_gate_up(const Dims& dm, int64_t T) {
   static const int bf16_bn[] = {16, 32, 64, 96, 128, 160, 192, 224, 256};
   static const int fp8_bn[] = {16, 32, 64, 96};
-  const double want = SMOE_BN_FACTOR * static_cast<double>(T) * dm.k / dm.E;
+  const double want = SMOE_BN_FACTOR * rows_per_group(dm, T);
   GemmPlan p;
   p.bn = dm.fp8 ? pick_bn(want, fp8_bn, 4) : pick_bn(want, bf16_bn, 9);
   p.na = 2;
@@ -61,7 +67,7 @@ GemmPlan plan_gate_up(const Dims& dm, int64_t T) {
 GemmPlan plan_down(const Dims& dm, int64_t T) {
   static const int bf16_bn[] = {16, 32, 64, 96, 128, 160, 192, 224, 256};
   static const int fp8_bn[] = {16, 32, 64, 128, 192};
-  const double want = SMOE_BN_FACTOR * static_cast<double>(T) * dm.k / dm.E;
+  const double want = SMOE_BN_FACTOR * rows_per_group(dm, T);
   GemmPlan p;
   p.bn = dm.fp8 ? pick_bn(want, fp8_bn, 5) : pick_bn(want, bf16_bn, 9);
   p.pair = !dm.fp8 && pair_bn_supported(p.bn) && dm.d % 256 == 0 && dm.f % 128 == 0;

@@ -117,6 +117,28 @@ def pin_layer_vs_brute_fp8(orc):
         np.testing.assert_allclose(y[t], yb, rtol=1e-9, atol=1e-12)
 
 
+def pin_dense_ffn_vs_brute(orc):
+    """The dense FFN (no router) equals the scalar-loop SwiGLU MLP, BF16 and
+    FP8 (d != i so a transposed operand cannot pass), and the layer's combine
+    with no routed experts (k = 0) and that MLP as its shared expert gives the
+    same y."""
+    T, d, i = 3, 24, 40
+    x, _, _, _, sh = small_layer(21, T, d, i, 1, 1)
+    mats = {"gate": sh[0], "up": sh[1], "down": sh[2]}
+    y = orc.dense_ffn(x, mats, "bf16")
+    for t in range(T):
+        np.testing.assert_allclose(y[t], brute.expert_token(x[t], *sh), rtol=1e-10, atol=1e-12)
+    yc = orc.experts_combine(x, np.zeros((T, 0), np.int64), np.zeros((T, 0)), None,
+                             lambda: mats, "bf16", 1)
+    np.testing.assert_array_equal(yc, y)
+    x8, _, _, _, sh8 = fp8_small_layer(22, T=2, d=256, f=128, E=1, k=1)
+    y8 = orc.dense_ffn(x8, sh8, "fp8")
+    shd = tuple(_dequant_scalar(sh8[n], sh8[n + "_scale"]) for n in ("gate", "up", "down"))
+    for t in range(2):
+        np.testing.assert_allclose(y8[t], brute.expert_token(x8[t], *shd, fp8=True), rtol=1e-9,
+                                   atol=1e-12)
+
+
 def pin_weights_sum(orc):
     """norm_topk_prob then routed_scaling_factor: the k weights of every token
     are positive and sum to 2.827."""
@@ -244,4 +266,4 @@ def pin_fp8_exact_grid(orc):
 ALL_PINS = [pin_route_vs_brute, pin_layer_vs_brute_bf16, pin_layer_vs_brute_fp8,
             pin_weights_sum, pin_bias_selects_only, pin_k_equals_E,
             pin_identical_experts_closed_form, pin_textbook_values, pin_printed_counts,
-            pin_act_quant, pin_fp8_exact_grid]
+            pin_act_quant, pin_fp8_exact_grid, pin_dense_ffn_vs_brute]

@@ -73,6 +73,21 @@ def test_create_rejects_bad_configs_before_touching_a_device(smoe, field, value,
     assert ei.value.status == getattr(smoe, expect)
 
 
+@pytest.mark.parametrize("E,k,ns,expect", [
+    (0, 8, 9, "MOE_ERR_INVALID_ARG"),   # no routed experts, yet k > 0
+    (0, 0, 0, "MOE_ERR_INVALID_ARG"),   # no routed and no shared experts: no layer
+    (384, 0, 1, "MOE_ERR_INVALID_ARG"),  # routed experts need k >= 1
+    (0, 0, 17, "MOE_ERR_UNSUPPORTED"),  # shared MLP wider than 16 x f
+])
+def test_dense_layer_configs_are_checked_before_touching_a_device(smoe, E, k, ns, expect):
+    """n_routed_experts = 0 (a dense FFN: the shared MLP alone) is a valid
+    layer only with num_experts_per_tok = 0 and 1..16 shared groups."""
+    c = smoe.moe_config_init_k2(n_routed_experts=E, num_experts_per_tok=k, n_shared_experts=ns)
+    with pytest.raises(smoe.MoeError) as ei:
+        smoe.moe_create(c, 0)
+    assert ei.value.status == getattr(smoe, expect)
+
+
 def test_null_handle_calls_are_rejected(smoe):
     lib = ctypes.CDLL(smoe.LIB_PATH)
     lib.moe_forward.restype = ctypes.c_int
