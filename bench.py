@@ -18,7 +18,10 @@ N > 1 runs one independent replica per GPU (data parallel over token
 batches; the layer has no exchange step at one GPU per replica), so the
 scaling is weak and the value is the tokens of all ranks / the slowest rank's
 time. Timing: CUDA events on the launch stream, W warm-up steps, then K
-steps between a barrier + synchronize on both sides; max over ranks. The
+plain forwards (as a caller runs them) between a barrier + synchronize on
+both sides; max over ranks. The phase times and the dominant kernel's
+roofline come from a further run of the same forwards with the library's
+per-phase events. The
 weights streamed per step (25-34 GB BF16) are far larger than the 126 MB L2,
 so no flush is needed between steps.
 
@@ -325,7 +328,8 @@ def run_native(args, wl):
         smoe.moe_forward(h, x, y)
     torch.cuda.synchronize()
 
-    smoe.moe_profile_enable(h, args.steps)
+    # the timed steps: plain forwards, as a caller runs them (the library
+    # replays them as a CUDA graph from the second call on)
     n0 = smoe.moe_launch_count(h)
     clocks = ClockSampler(local)
     clocks.start()
@@ -343,7 +347,14 @@ def run_native(args, wl):
     clk = clocks.stop()
     launches = smoe.moe_launch_count(h) - n0
     ms_total = e0.elapsed_time(e1)
-    phases = np.array(smoe.moe_profile_read(h, args.steps))
+    # then the same forwards with the library's per-phase events (launched one
+    # by one), for the phase times and the dominant kernel's roofline
+    n_prof = min(args.steps, 50)
+    smoe.moe_profile_enable(h, n_prof)
+    for _ in range(n_prof):
+        smoe.moe_forward(h, x, y)
+    torch.cuda.synchronize()
+    phases = np.array(smoe.moe_profile_read(h, n_prof))
     smoe.moe_profile_enable(h, 0)
     st = smoe.moe_get_device_status(h)
     if st:

@@ -174,6 +174,15 @@ void free_all(moe_handle* h) {
   if (h->up) cudaStreamDestroy(h->up);
   if (h->down) cudaStreamDestroy(h->down);
   h->up = h->down = nullptr;
+  for (auto& g : h->graphs) {
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+    g = moe_handle::Graph{};
+  }
+  if (h->cap) cudaStreamDestroy(h->cap);
+  if (h->ev_in) cudaEventDestroy(h->ev_in);
+  if (h->ev_out) cudaEventDestroy(h->ev_out);
+  h->cap = nullptr;
+  h->ev_in = h->ev_out = nullptr;
   for (cudaEvent_t e : h->prof_events) cudaEventDestroy(e);
   h->prof_events.clear();
 }
@@ -297,7 +306,10 @@ moe_status_t moe_create(const moe_config_t* cfg, int device, moe_handle_t** out)
   }
   if (rc == MOE_OK) {
     bool ok = cudaStreamCreateWithFlags(&h->up, cudaStreamNonBlocking) == cudaSuccess &&
-              cudaStreamCreateWithFlags(&h->down, cudaStreamNonBlocking) == cudaSuccess;
+              cudaStreamCreateWithFlags(&h->down, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&h->ev_in, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&h->ev_out, cudaEventDisableTiming) == cudaSuccess;
     for (int b = 0; b < 2 && ok; ++b)
       ok = cudaEventCreateWithFlags(&h->ev_x[b], cudaEventDisableTiming) == cudaSuccess &&
            cudaEventCreateWithFlags(&h->ev_fwd[b], cudaEventDisableTiming) == cudaSuccess &&
@@ -438,6 +450,12 @@ static moe_status_t read_status(moe_handle* h, cudaStream_t s, uint32_t* flags) 
   return MOE_OK;
 }
 
+namespace {
+moe_status_t launch_forward(moe_handle* h, const void* x, int64_t T, void* y,
+                            const moe_forward_opts_t* opts, cudaStream_t s, cudaEvent_t* ev);
+moe_status_t forward_graphed(moe_handle* h, const void* x, int64_t T, void* y, cudaStream_t s);
+}  // namespace
+
 moe_status_t moe_forward(moe_handle_t* h, const void* x, int64_t T, void* y,
                          const moe_forward_opts_t* opts, void* stream) {
   if (h == nullptr) return MOE_ERR_INVALID_ARG;
@@ -456,11 +474,21 @@ moe_status_t moe_forward(moe_handle_t* h, const void* x, int64_t T, void* y,
   DeviceGuard guard(h->device);
   if (!guard.ok) return fail(h, MOE_ERR_CUDA, "cudaSetDevice failed");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int Ti = static_cast<int>(T);
-
   cudaEvent_t* ev = nullptr;
   if (h->prof_next < h->prof_cap)
     ev = h->prof_events.data() + static_cast<size_t>(h->prof_next) * (MOE_NUM_PHASES + 1);
+  if (opts == nullptr && ev == nullptr) return forward_graphed(h, x, T, y, s);
+  return launch_forward(h, x, T, y, opts, s, ev);
+}
+
+namespace {
+
+// The launch sequence of one forward on stream s (ev: per-phase events, or
+// NULL).
+moe_status_t launch_forward(moe_handle* h, const void* x, int64_t T, void* y,
+                            const moe_forward_opts_t* opts, cudaStream_t s, cudaEvent_t* ev) {
+  const Dims& dm = h->dims;
+  const int Ti = static_cast<int>(T);
   auto mark = [&](int i) {
     if (ev) cudaEventRecord(ev[i], s);
   };
@@ -526,6 +554,60 @@ moe_status_t moe_forward(moe_handle_t* h, const void* x, int64_t T, void* y,
   }
   return MOE_OK;
 }
+
+// A forward without options or profiling, as a CUDA graph: at small T the
+// layer is a chain of short kernels and the launches themselves are a large
+// part of the step. The first call with a given (T, x, y) launches directly
+// (which also does each kernel's one-time attribute setup); the second
+// captures the same launch sequence on the handle's capture stream, and every
+// later call replays it there, ordered after the caller's stream by an event
+// and with the caller's stream waiting for it.
+moe_status_t forward_graphed(moe_handle* h, const void* x, int64_t T, void* y, cudaStream_t s) {
+  moe_handle::Graph* g = nullptr;
+  for (auto& e : h->graphs)
+    if (e.T == T && e.x == x && e.y == y) g = &e;
+  if (g == nullptr) {  // first sight: remember it, launch directly
+    moe_handle::Graph* slot = &h->graphs[0];
+    for (auto& e : h->graphs)
+      if (e.last_use < slot->last_use) slot = &e;
+    if (slot->exec) cudaGraphExecDestroy(slot->exec);
+    *slot = moe_handle::Graph{};
+    slot->T = T;
+    slot->x = x;
+    slot->y = y;
+    slot->last_use = ++h->graph_clock;
+    return launch_forward(h, x, T, y, nullptr, s, nullptr);
+  }
+  g->last_use = ++h->graph_clock;
+  if (g->exec == nullptr && !g->failed) {  // second sight: capture
+    const int64_t n0 = h->launches;
+    cudaGraph_t graph = nullptr;
+    bool ok = cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+    moe_status_t st = ok ? launch_forward(h, x, T, y, nullptr, h->cap, nullptr) : MOE_ERR_CUDA;
+    if (ok) ok = cudaStreamEndCapture(h->cap, &graph) == cudaSuccess && st == MOE_OK;
+    if (ok) ok = cudaGraphInstantiate(&g->exec, graph, 0) == cudaSuccess;
+    if (graph) cudaGraphDestroy(graph);
+    const int64_t captured = h->launches - n0;  // kernels in the graph
+    h->launches = n0;
+    if (!ok) {  // run without a graph from now on for this key
+      g->failed = true;
+      g->exec = nullptr;
+      cudaGetLastError();
+    } else {
+      g->launches = captured;
+    }
+  }
+  if (g->exec == nullptr) return launch_forward(h, x, T, y, nullptr, s, nullptr);
+  CUDA_TRY(h, cudaEventRecord(h->ev_in, s), "graph order");
+  CUDA_TRY(h, cudaStreamWaitEvent(h->cap, h->ev_in, 0), "graph order");
+  CUDA_TRY(h, cudaGraphLaunch(g->exec, h->cap), "graph launch");
+  CUDA_TRY(h, cudaEventRecord(h->ev_out, h->cap), "graph order");
+  CUDA_TRY(h, cudaStreamWaitEvent(s, h->ev_out, 0), "graph order");
+  h->launches += g->launches;
+  return MOE_OK;
+}
+
+}  // namespace
 
 moe_status_t moe_forward_host_async(moe_handle_t* h, const void* x_host, int64_t T, void* y_host,
                                     const moe_forward_opts_t* opts, void* stream) {

@@ -95,6 +95,21 @@ struct moe_handle {
   cudaStream_t up = nullptr, down = nullptr;
   cudaEvent_t ev_x[2] = {}, ev_fwd[2] = {}, ev_y[2] = {};
   uint64_t host_calls = 0;
+  // forwards replayed as CUDA graphs, keyed by (T, x, y); captured and
+  // replayed on `cap`, ordered against the caller's stream by ev_in / ev_out
+  struct Graph {
+    int64_t T = 0;
+    const void* x = nullptr;
+    void* y = nullptr;
+    cudaGraphExec_t exec = nullptr;
+    int64_t launches = 0;  // kernels in the graph
+    uint64_t last_use = 0;
+    bool failed = false;
+  };
+  Graph graphs[8];
+  uint64_t graph_clock = 0;
+  cudaStream_t cap = nullptr;
+  cudaEvent_t ev_in = nullptr, ev_out = nullptr;
 };
 
 namespace smoe {

@@ -185,6 +185,27 @@ def test_host_pipeline_matches_device(smoe, tiny):
     assert torch.equal(yone, want[1])
 
 
+def test_repeated_forwards_replay_a_graph(smoe, tiny):
+    """From the second forward with the same (T, x, y) and no options the
+    library replays a captured CUDA graph: each result follows the current
+    contents of x in the same buffers, equal to a direct forward (one with
+    options, which never uses a graph), and the launch count still counts
+    the graph's kernels."""
+    layer, h = tiny
+    scales = (1.0, 0.5, 2.0, -1.0, 0.25)
+    want = [gu.run(smoe, h, layer, (layer.x[:64] * c).contiguous())[0].clone() for c in scales]
+    x = torch.empty_like(layer.x[:64])
+    y = torch.empty_like(x)
+    n0 = smoe.moe_launch_count(h)
+    for i, c in enumerate(scales):
+        x.copy_(layer.x[:64] * c)
+        smoe.moe_forward(h, x, y)
+        torch.cuda.synchronize()
+        assert torch.equal(y, want[i]), i
+    assert smoe.moe_launch_count(h) - n0 == len(scales) * 7
+    assert smoe.moe_get_device_status(h) == 0
+
+
 def test_profile_phases(smoe, tiny):
     layer, h = tiny
     smoe.moe_profile_enable(h, 3)
