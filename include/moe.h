@@ -157,7 +157,14 @@ moe_status_t moe_load_weights(moe_handle_t* h, const moe_weights_t* w, void* str
 /* y = MoE(x) for T tokens. x: device BF16 [T, d]; y: device BF16 [T, d]
  * (must not overlap x). T = 0 is a no-op. T > max_tokens is
  * MOE_ERR_INVALID_ARG. Asynchronous on `stream` unless opts->flags has
- * MOE_FLAG_SYNC_CHECK. opts may be NULL. */
+ * MOE_FLAG_SYNC_CHECK. opts may be NULL.
+ * A forward with opts == NULL and profiling off is captured, on its second
+ * call with the same (T, x, y), as a CUDA graph and replayed from then on
+ * (eight such shapes are kept, least recently used replaced): it then runs
+ * on a stream of the handle, after the work already on `stream`, and
+ * `stream` waits for it, so the ordering seen by the caller is unchanged. The
+ * graph reads x and writes y at run time, so their contents may change
+ * between calls; buffers at the same addresses must stay allocated. */
 moe_status_t moe_forward(moe_handle_t* h, const void* x, int64_t T, void* y,
                          const moe_forward_opts_t* opts, void* stream);
 
