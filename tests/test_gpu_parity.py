@@ -236,6 +236,29 @@ def test_k2_decode_T64(smoe, k2):
     _check(gu.compare(layer, y, ids, w, tokens=toks, x=x))
 
 
+def test_k2_all_tokens_on_eight_experts(smoe, k2):
+    """Maximal imbalance: every token forced onto experts 0..7 (376 experts
+    empty, 2048 rows each for the 8, cut into many row tiles): ids as forced,
+    weights from the oracle's scores for those ids, outputs of sampled tokens
+    against the oracle with the same ids and weights."""
+    layer, h = k2
+    T, k = 2048, 8
+    x = layer.x[:T].contiguous()
+    ids = np.tile(np.arange(k, dtype=np.int32), (T, 1))
+    forced = torch.from_numpy(ids).cuda()
+    y, gids, gw = gu.run(smoe, h, layer, x, forced=forced)
+    assert np.array_equal(gu.to_np(gids), ids)
+    r = gu.oracle_route(layer, x)
+    sc = np.take_along_axis(r.scores.astype(np.float64), ids.astype(np.int64), axis=1)
+    w = 2.827 * sc / sc.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(gu.to_np(gw), w, rtol=1e-5)
+    toks = np.random.default_rng(3).choice(T, 6, replace=False)
+    yo = gu.oracle_outputs(layer, ids.astype(np.int64), w, toks, x)
+    err = np.max(np.abs(gu.to_np(y).astype(np.float64)[toks] - yo)) / np.max(np.abs(yo))
+    assert err <= gu.TOL["bf16"], err
+    assert smoe.moe_get_device_status(h) == 0
+
+
 def test_k2_prefill_T8192(smoe, k2):
     layer, h = k2
     y, ids, w = gu.run(smoe, h, layer)
