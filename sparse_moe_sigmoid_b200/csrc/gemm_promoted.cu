@@ -97,6 +97,27 @@ struct PromCfg {
   }
 };
 
+// Two fp32 operations per instruction (sm_100 packed fp32): the same IEEE
+// round-to-nearest results as two scalar ones. The promotion's arithmetic is
+// the FP8 GEMMs' critical path at large T (measured: ~1000 cycles per 128-K
+// block against ~400 of MMA work).
+__device__ __forceinline__ void fma2(float& a0, float& a1, float x0, float x1, float c0,
+                                     float c1) {
+  asm("{\n\t.reg .b64 A, X, C;\n\t"
+      "mov.b64 A, {%0, %1};\n\tmov.b64 X, {%2, %3};\n\tmov.b64 C, {%4, %5};\n\t"
+      "fma.rn.f32x2 A, X, C, A;\n\tmov.b64 {%0, %1}, A;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(x0), "f"(x1), "f"(c0), "f"(c1));
+}
+
+__device__ __forceinline__ void mul2(float& d0, float& d1, float x0, float x1, float y0, float y1) {
+  asm("{\n\t.reg .b64 D, X, Y;\n\t"
+      "mov.b64 X, {%2, %3};\n\tmov.b64 Y, {%4, %5};\n\t"
+      "mul.rn.f32x2 D, X, Y;\n\tmov.b64 {%0, %1}, D;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(x0), "f"(x1), "f"(y0), "f"(y1));
+}
+
 // registers per thread for the one CTA per SM: the register file is four
 // 16K-register slices, one per scheduler, and a block's warps are spread over
 // them, so a slice holds ceil(warps / 4) warps; rounded down to the
@@ -332,16 +353,34 @@ __global__ void __maxnreg__(prom_regs<NPG>())
 #pragma unroll
           for (int c = 0; c < C::kBatch / 16; ++c) {
             if (c_begin + b0 + c * 16 < un.nvalid) {
+              if (FP8) {
+                // acc += partial * (s_w * s_x[row]): four activation scales per
+                // 16-byte load (all lanes read the same address), then pairs
+                // of columns per packed multiply and multiply-add
 #pragma unroll
-              for (int jj = c * 16; jj < c * 16 + 16; ++jj) {
-                const int j = b0 + jj;
-                if (FP8) {
-                  const float s = sa[j];
-                  acc0[j] = fmaf(__uint_as_float(g[jj]), sw0 * s, acc0[j]);
-                  if (C::kTwoA) acc1[j] = fmaf(__uint_as_float(v[jj]), sw1 * s, acc1[j]);
-                } else {
-                  acc0[j] += __uint_as_float(g[jj]);
+                for (int jj = c * 16; jj < c * 16 + 16; jj += 4) {
+                  const int j = b0 + jj;
+                  const float4 s4 = *reinterpret_cast<const float4*>(sa + j);
+                  float c00, c01, c02, c03;
+                  mul2(c00, c01, sw0, sw0, s4.x, s4.y);
+                  mul2(c02, c03, sw0, sw0, s4.z, s4.w);
+                  fma2(acc0[j], acc0[j + 1], __uint_as_float(g[jj]), __uint_as_float(g[jj + 1]),
+                       c00, c01);
+                  fma2(acc0[j + 2], acc0[j + 3], __uint_as_float(g[jj + 2]),
+                       __uint_as_float(g[jj + 3]), c02, c03);
+                  if (C::kTwoA) {
+                    float c10, c11, c12, c13;
+                    mul2(c10, c11, sw1, sw1, s4.x, s4.y);
+                    mul2(c12, c13, sw1, sw1, s4.z, s4.w);
+                    fma2(acc1[j], acc1[j + 1], __uint_as_float(v[jj]), __uint_as_float(v[jj + 1]),
+                         c10, c11);
+                    fma2(acc1[j + 2], acc1[j + 3], __uint_as_float(v[jj + 2]),
+                         __uint_as_float(v[jj + 3]), c12, c13);
+                  }
                 }
+              } else {
+#pragma unroll
+                for (int jj = c * 16; jj < c * 16 + 16; ++jj) acc0[b0 + jj] += __uint_as_float(g[jj]);
               }
             }
           }
