@@ -69,3 +69,21 @@ def test_algorithmic_counts_match_the_expert_size():
     assert a["layer"][0] - (385 * per_expert) == 384 * 7168 * 4 + 384 * 4 + 48 * 7168 * 4
     R = 48 * 9
     assert a["gemm_gate_up"][1] == 2 * R * 2 * 2048 * 7168
+
+
+def test_dense_workload_and_its_counts():
+    """K2's dense FFN layer: no router, 9 shared groups of 2048 (intermediate
+    18432); its algorithmic work is one 3 x 7168 x 18432 MLP over T rows."""
+    w = bench.workload("dense-T64")
+    s = w["shape"]
+    assert (w["T"], w["fmt"]) == (64, "bf16")
+    assert (s.n_routed_experts, s.num_experts_per_tok, s.n_shared_experts) == (0, 0, 9)
+    assert s.moe_intermediate_size * s.n_shared_experts == 18432
+    assert bench.workload("dense-fp8-T128")["fmt"] == "fp8"
+    T = 64
+    a = bench.algorithmic(s, T, "bf16", np.zeros((T, 0), np.int64))
+    assert a["U"] == 0
+    assert a["gemm_gate_up"][0] == 2 * 18432 * 7168 * 2 + T * 9 * (7168 + 2048) * 2
+    assert a["gemm_gate_up"][1] == 2 * T * 2 * 18432 * 7168
+    assert a["gemm_down"][1] == 2 * T * 18432 * 7168
+    assert a["layer"][1] == 2 * T * 3 * 18432 * 7168
