@@ -495,7 +495,9 @@ moe_status_t launch_forward(moe_handle* h, const void* x, int64_t T, void* y,
 
   const GemmPlan p1 = smoe::plan_gate_up(dm, T);
   const GemmPlan p2 = smoe::plan_down(dm, T);
-  const int splits = dm.E > 0 ? smoe::router_splits(dm, T, h->num_sms) : 0;
+  const int splits = dm.E == 0                       ? 0
+                     : T <= smoe::kRouterGemvMaxT ? 1  // the GEMV router: one slice
+                                                  : smoe::router_splits(dm, T, h->num_sms);
   const int32_t* forced = opts ? opts->forced_topk_ids : nullptr;
 
   mark(0);

@@ -18,6 +18,7 @@ constexpr int kMaxExperts = 512;
 constexpr int kRouterTile = 64;   // router tile: 64 tokens x 64 experts
 constexpr int kRouterKTile = 32;
 constexpr int kRouterMaxSplits = 32;
+constexpr int kRouterGemvMaxT = 8;  // up to this many tokens the logits are a GEMV (one slice)
 
 // Sizes derived from the config, fixed per handle.
 struct Dims {

@@ -261,8 +261,61 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
   }
 }
 
+// Few tokens (T <= kRouterGemvMaxT): the 64 x 64 tiles of router_logits_kernel
+// would hold one or a few valid tokens and need a split-K sum, so instead one
+// CTA per expert reads its router row once (float4 loads, 256 threads
+// striding K) and accumulates every token's dot product; the 8 warps' sums
+// are added in a fixed order (deterministic). One partial slice: splits = 1.
+__global__ void __launch_bounds__(256) router_gemv_kernel(const __nv_bfloat16* __restrict__ x,
+                                                          const float* __restrict__ W,
+                                                          float* __restrict__ part, int T, int E,
+                                                          int d) {
+  __shared__ float red[8][kRouterGemvMaxT];
+  const int e = blockIdx.x;
+  const float* w = W + (size_t)e * d;
+  float acc[kRouterGemvMaxT];
+#pragma unroll
+  for (int t = 0; t < kRouterGemvMaxT; ++t) acc[t] = 0.f;
+  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
+    const float4 wv = __ldg(reinterpret_cast<const float4*>(w + c));
+#pragma unroll
+    for (int t = 0; t < kRouterGemvMaxT; ++t) {
+      if (t < T) {
+        const uint2 raw = __ldg(reinterpret_cast<const uint2*>(x + (size_t)t * d + c));
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+        acc[t] = fmaf(a.x, wv.x, acc[t]);
+        acc[t] = fmaf(a.y, wv.y, acc[t]);
+        acc[t] = fmaf(b.x, wv.z, acc[t]);
+        acc[t] = fmaf(b.y, wv.w, acc[t]);
+      }
+    }
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int t = 0; t < kRouterGemvMaxT; ++t) {
+    float v = acc[t];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if (lane == 0) red[warp][t] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < T) {
+    float sum = 0.f;
+#pragma unroll
+    for (int w8 = 0; w8 < 8; ++w8) sum += red[w8][threadIdx.x];
+    part[(size_t)threadIdx.x * E + e] = sum;
+  }
+}
+
 cudaError_t launch_router_logits(moe_handle* h, const void* x, int T, int splits, cudaStream_t s) {
   const Dims& dm = h->dims;
+  if (T <= kRouterGemvMaxT) {  // the caller passes splits = 1 for these
+    router_gemv_kernel<<<dm.E, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), h->w.router,
+                                            h->ws.logits_part, T, dm.E, dm.d);
+    h->launches++;
+    return cudaGetLastError();
+  }
   dim3 grid((dm.E + kRouterTile - 1) / kRouterTile, (T + kRouterTile - 1) / kRouterTile, splits);
   router_logits_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), h->w.router,
                                             h->ws.logits_part, T, dm.E, dm.d,

@@ -270,7 +270,7 @@ def test_k2_prefill_T8192(smoe, k2):
 
 
 # ------------------------------------------------------------ router logits
-@pytest.mark.parametrize("T", [64, 512, 8192])
+@pytest.mark.parametrize("T", [4, 64, 512, 8192])
 def test_k2_router_logit_accuracy(smoe, k2, T):
     """Logits from the CUDA-core path (small T) and the tensor-core path
     (T >= 512, fp32 router weight split exactly into three BF16 parts)
