@@ -245,7 +245,7 @@ def algorithmic(shape, T, fmt, ids: np.ndarray):
     R = T * (k + ns)
     sb = lambda r, c: (r // 128) * (c // 128) * 4 if fmt == "fp8" else 0
     gate_up_bytes = G_used * 2 * (f * d * wb + sb(f, d)) + R * d * wb + R * f * wb
-    down_bytes = G_used * (d * f * wb + sb(d, f)) + R * f * wb + R * d * 4
+    down_bytes = G_used * (d * f * wb + sb(d, f)) + R * f * wb + R * d * 2  # BF16 row outputs
     if fmt == "fp8":
         gate_up_bytes += R * (d // 128) * 4 + R * (f // 128) * 4
         down_bytes += R * (f // 128) * 4

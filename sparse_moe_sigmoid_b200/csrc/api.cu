@@ -298,7 +298,7 @@ moe_status_t moe_create(const moe_config_t* cfg, int device, moe_handle_t** out)
     A(&h->ws.xs, Rm * (d / 128) * 4, "x scales");
     A(&h->ws.hs, Rm * (f / 128) * 4, "h scales");
   }
-  A(&h->ws.out, Rm * d * 4, "expert outputs");
+  A(&h->ws.out, Rm * d * 2, "expert outputs");
   A(&h->ws.status, 4, "status");
   for (int b = 0; b < 2; ++b) {
     A(&h->ws.x_stage[b], Tm * d * 2, "x staging");

@@ -20,7 +20,8 @@
 //   per 128 columns s = amax/448 and q = e4m3(x/s), both divisions
 //   correctly rounded, conversion nearest-even and saturating.
 // combine_kernel: y[t] = sum_j w[t,j] * out[row(t,j)] + sum_s out[shared
-//   row(s,t)] in fp32, in slot order, rounded once to BF16.
+//   row(s,t)] over the BF16 per-row outputs, summed in fp32 in slot order and
+//   rounded once to BF16.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
@@ -296,47 +297,49 @@ cudaError_t launch_dispatch(moe_handle* h, const void* x, int T, cudaStream_t s)
 }
 
 // ------------------------------------------------------------------ combine
-__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ out,
-                                                      const int32_t* __restrict__ pair_row,
-                                                      const float* __restrict__ wts,
-                                                      const int32_t* __restrict__ offsets, int T,
-                                                      int d, int k, int E, int ns,
-                                                      __nv_bfloat16* __restrict__ y) {
+// 8 columns per thread: one 16-byte load per expert row, one 16-byte store.
+constexpr int kCombineThreads = 128;
+
+__device__ __forceinline__ void add_row8(float (&acc)[8], const uint16_t* p, float w) {
+  const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {  // BF16 -> fp32 is exact: the bits move up by 16
+    acc[2 * i] = fmaf(w, __uint_as_float(u[i] << 16), acc[2 * i]);
+    acc[2 * i + 1] = fmaf(w, __uint_as_float(u[i] & 0xFFFF0000u), acc[2 * i + 1]);
+  }
+}
+
+__global__ void __launch_bounds__(kCombineThreads)
+    combine_kernel(const uint16_t* __restrict__ out, const int32_t* __restrict__ pair_row,
+                   const float* __restrict__ wts, const int32_t* __restrict__ offsets, int T, int d,
+                   int k, int E, int ns, __nv_bfloat16* __restrict__ y) {
   const int t = blockIdx.x;
-  const int c = (blockIdx.y * blockDim.x + threadIdx.x) * 4;
+  const int c = (blockIdx.y * blockDim.x + threadIdx.x) * 8;
   if (c >= d) return;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
   for (int j = 0; j < k; ++j) {
     const int row = pair_row[(size_t)t * k + j];
-    const float w = wts[(size_t)t * k + j];
-    const float4 v = __ldg(reinterpret_cast<const float4*>(out + (size_t)row * d + c));
-    acc.x = fmaf(w, v.x, acc.x);
-    acc.y = fmaf(w, v.y, acc.y);
-    acc.z = fmaf(w, v.z, acc.z);
-    acc.w = fmaf(w, v.w, acc.w);
+    add_row8(acc, out + (size_t)row * d + c, wts[(size_t)t * k + j]);
   }
-  for (int s = 0; s < ns; ++s) {
-    const int row = offsets[E + s] + t;
-    const float4 v = __ldg(reinterpret_cast<const float4*>(out + (size_t)row * d + c));
-    acc.x += v.x;
-    acc.y += v.y;
-    acc.z += v.z;
-    acc.w += v.w;
+  for (int s = 0; s < ns; ++s) add_row8(acc, out + (size_t)(offsets[E + s] + t) * d + c, 1.f);
+  uint32_t pk[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+    pk[i] = *reinterpret_cast<uint32_t*>(&b);
   }
-  __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-  __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-  uint2 pk;
-  pk.x = *reinterpret_cast<uint32_t*>(&lo);
-  pk.y = *reinterpret_cast<uint32_t*>(&hi);
-  *reinterpret_cast<uint2*>(y + (size_t)t * d + c) = pk;
+  *reinterpret_cast<uint4*>(y + (size_t)t * d + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
 }
 
 cudaError_t launch_combine(moe_handle* h, void* y, int T, cudaStream_t s) {
   const Dims& dm = h->dims;
-  dim3 grid(T, (dm.d / 4 + 255) / 256);
-  combine_kernel<<<grid, 256, 0, s>>>(h->ws.out, h->ws.pair_row, h->ws.wts, h->ws.offsets, T,
-                                      dm.d, dm.k, dm.E, dm.ns,
-                                      static_cast<__nv_bfloat16*>(y));
+  dim3 grid(T, (dm.d / 8 + kCombineThreads - 1) / kCombineThreads);
+  combine_kernel<<<grid, kCombineThreads, 0, s>>>(h->ws.out, h->ws.pair_row, h->ws.wts,
+                                                  h->ws.offsets, T, dm.d, dm.k, dm.E, dm.ns,
+                                                  static_cast<__nv_bfloat16*>(y));
   h->launches++;
   return cudaGetLastError();
 }

@@ -23,7 +23,7 @@
 //               finished accumulators to the epilogue.
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator (TMEM lane = output
 //               feature, column = row), then SwiGLU and a BF16 store of h, or
-//               an fp32 store of the down projection's per-row output. The
+//               a BF16 store of the down projection's per-row output. The
 //               second accumulator buffer lets the next tile's MMAs run
 //               meanwhile.
 // Every wait is bounded (2 s); a wait that runs out sets
@@ -229,9 +229,10 @@ __global__ void __launch_bounds__(192, 1)
               const float hv = gv / (1.f + expf(-gv)) * uv;
               static_cast<__nv_bfloat16*>(args.out)[row * args.ld + feat] = __float2bfloat16_rn(hv);
             } else {
-              float* o = static_cast<float*>(args.out) + row * args.ld;
-              if (feat < args.m_valid) o[feat] = __uint_as_float(g[j]);
-              if (NA == 2 && feat + 128 < args.m_valid) o[feat + 128] = __uint_as_float(v[j]);
+              __nv_bfloat16* o = static_cast<__nv_bfloat16*>(args.out) + row * args.ld;
+              if (feat < args.m_valid) o[feat] = __float2bfloat16_rn(__uint_as_float(g[j]));
+              if (NA == 2 && feat + 128 < args.m_valid)
+                o[feat + 128] = __float2bfloat16_rn(__uint_as_float(v[j]));
             }
           }
         }

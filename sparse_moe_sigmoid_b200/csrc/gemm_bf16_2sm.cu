@@ -16,7 +16,7 @@
 //     barriers of both CTAs (and, per unit, to both `tfull` barriers);
 //   each CTA's eight epilogue warps (two per TMEM lane quarter, taking
 //     alternate 16-column chunks) drain their own TMEM (SwiGLU + BF16 h, or
-//     the fp32 per-row output) and signal the even CTA's `tempty` barrier.
+//     the per-row output, rounded to BF16) and signal the even CTA's `tempty` barrier.
 //
 // Shared-memory fill from L2, not the tensor core, bounds these kernels at
 // prefill sizes (measured: as fast with the MMAs removed), so each unit loads
@@ -383,7 +383,8 @@ __global__ void __maxnreg__(kPairRegs)
                 const float hv = silu_mul(__uint_as_float(g[j]), __uint_as_float(v[j]));
                 static_cast<__nv_bfloat16*>(args.out)[row * args.ld + feat] = __float2bfloat16_rn(hv);
               } else if (feat < args.m_valid) {
-                static_cast<float*>(args.out)[row * args.ld + feat] = __uint_as_float(g[j]);
+                static_cast<__nv_bfloat16*>(args.out)[row * args.ld + feat] =
+                    __float2bfloat16_rn(__uint_as_float(g[j]));
               }
             }
           }

@@ -30,7 +30,7 @@ struct GemmArgs {
   int m_tiles;
   int k_blocks;
   int bn;
-  void* out;                 // gate/up: h [R][ld]; down: fp32 out [R][ld]
+  void* out;                 // gate/up: h [R][ld]; down: BF16 out [R][ld]; router: fp32
   int ld;
   float* out_scale;          // FP8 gate/up: h scales [R][f/128]
   const float* w_scale0;     // FP8: weight block scales of A0 [G][m_tiles][k_blocks]
@@ -47,6 +47,7 @@ struct GemmArgs {
                              // covers k-blocks [s, s+1) * k_blocks / ksplit and writes its
                              // partial result at out + s * split_stride elements
   size_t split_stride;
+  int out_bf16;               // promoted GEMM, plain mode: outputs stored BF16 (else fp32)
 };
 
 __device__ __forceinline__ int total_units_of(const GemmArgs& a, int BN) {

@@ -21,7 +21,7 @@
 // 128 features, which is exactly this tile's 128 features: s_h = amax/448,
 // q = e4m3(h / s_h) (correctly rounded divisions, nearest-even saturating
 // conversion), written with its scale for the down GEMM.
-// Down epilogue: the promoted fp32 row outputs.
+// Down epilogue: the promoted fp32 row outputs, rounded to BF16 once.
 //
 // The same kernel with BF16 operands and no scales computes the router
 // logits on the tensor cores (launch_router_gemm below): there the point of
@@ -38,6 +38,7 @@
 // work per thread and allow tiles of 128 rows with gate and up, 256 without).
 // The shared-memory ring's depth is set at launch from what the scale
 // staging of the actual K leaves free.
+#include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <stdio.h>
 
@@ -57,7 +58,7 @@ constexpr int kPromSmemBudget = 227 * 1024 - 2048;
 // Otherwise BF16 operands, 64 K per stage, no scales.
 // DUAL (FP8 down projection, short row tiles): two consecutive 128-feature
 // weight tiles per unit, loaded, multiplied and promoted like gate and up,
-// both stored as fp32 outputs, so that a stage carries two weight tiles.
+// both stored as row outputs, so that a stage carries two weight tiles.
 template <int BN, bool GATED, bool FP8, int NPG, bool DUAL = false>
 struct PromCfg {
   static constexpr bool kTwoA = GATED || DUAL;
@@ -425,19 +426,23 @@ __global__ void __maxnreg__(prom_regs<NPG>())
           }
         }
       } else {
-        float* out = static_cast<float*>(args.out) + un.split * args.split_stride;
+        // expert outputs (down) in BF16; router logit partials in fp32
+        auto put = [&](size_t i, float v) {
+          if (args.out_bf16) static_cast<__nv_bfloat16*>(args.out)[i] = __float2bfloat16_rn(v);
+          else static_cast<float*>(args.out)[un.split * args.split_stride + i] = v;
+        };
         const int f0 = DUAL ? un.mt * 256 + q * 32 + lane : feat;
         if (f0 < args.m_valid) {
 #pragma unroll
           for (int j = 0; j < C::kCols; ++j)
             if (c_begin + j < un.nvalid)
-              out[static_cast<size_t>(un.row0 + c_begin + j) * args.ld + f0] = acc0[j];
+              put(static_cast<size_t>(un.row0 + c_begin + j) * args.ld + f0, acc0[j]);
         }
         if (DUAL && f0 + 128 < args.m_valid) {
 #pragma unroll
           for (int j = 0; j < C::kCols; ++j)
             if (c_begin + j < un.nvalid)
-              out[static_cast<size_t>(un.row0 + c_begin + j) * args.ld + f0 + 128] = acc1[j];
+              put(static_cast<size_t>(un.row0 + c_begin + j) * args.ld + f0 + 128, acc1[j]);
         }
       }
     }
@@ -525,6 +530,7 @@ cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaSt
     }
   }
   a.out = h->ws.out;
+  a.out_bf16 = 1;
   a.ld = dm.d;
   a.w_scale0 = h->w.down_s;
   a.w_scale1 = h->w.down_s;

@@ -52,7 +52,7 @@ struct Workspace {
   float* xs = nullptr;            // [Rmax][d/128] FP8 activation scales
   void* hbuf = nullptr;           // [Rmax][f] SwiGLU output, BF16 or e4m3
   float* hs = nullptr;            // [Rmax][f/128] FP8 scales of h
-  float* out = nullptr;           // [Rmax][d] fp32 per-row expert outputs
+  uint16_t* out = nullptr;        // [Rmax][d] BF16 per-row expert outputs
   uint32_t* status = nullptr;     // device status word
   void* x_stage[2] = {};          // [Tmax][d] BF16 staging of the host entry points, used in turn
   void* y_stage[2] = {};          // [Tmax][d]
