@@ -87,3 +87,29 @@ def test_dense_workload_and_its_counts():
     assert a["gemm_gate_up"][1] == 2 * T * 2 * 18432 * 7168
     assert a["gemm_down"][1] == 2 * T * 18432 * 7168
     assert a["layer"][1] == 2 * T * 3 * 18432 * 7168
+
+
+def test_reference_arm_prints_the_contract_line(capsys):
+    """`bench.py --impl reference` (the float64 oracle on the host cores) prints
+    one JSON line with the bench keys, impl "reference", a cpu_baseline of
+    kind "oracle" equal to the line's value, and an e2e that moves no bytes."""
+    import json
+    bench.main(["--impl", "reference", "--steps", "1", "--warmup", "0", "--tokens", "8",
+                "--experts", "16"])
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in j, key
+    assert j["impl"] == "reference" and j["dtype"] == "f64" and j["n_gpus"] == 1
+    assert j["steps"] == 1 and j["warmup"] == 0 and j["higher_is_better"] is True
+    assert j["value"] > 0 and j["unit"] == "tokens/s"
+    cb = j["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == j["value"] and cb["cores"] >= 1
+    assert "tokens" in cb["sample"]
+    e2e = j["e2e"]
+    assert e2e["value"] == j["value"] and e2e["unit"] == j["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+    assert j["config"]["tokens"] == 8 and j["config"]["n_routed_experts"] == 16
