@@ -86,6 +86,8 @@ def test_dense_workload_and_its_counts():
     assert a["gemm_gate_up"][0] == 2 * 18432 * 7168 * 2 + T * 9 * (7168 + 2048) * 2
     assert a["gemm_gate_up"][1] == 2 * T * 2 * 18432 * 7168
     assert a["gemm_down"][1] == 2 * T * 18432 * 7168
+    # down: the weights once, h rows in, BF16 per-row outputs out
+    assert a["gemm_down"][0] == 18432 * 7168 * 2 + T * 9 * 2048 * 2 + T * 9 * 7168 * 2
     assert a["layer"][1] == 2 * T * 3 * 18432 * 7168
 
 
