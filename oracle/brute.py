@@ -34,21 +34,41 @@ def _sig(z: float) -> float:
     return 1.0 / (1.0 + math.exp(-z))
 
 
-def route_token(xt, Wg, bias, k, scale=2.827, norm=True):
-    """Returns (ids list, weights list) for one token."""
+def _best(vals, allowed, taken):
+    """Index of the largest allowed, untaken value; ties to the lower index."""
+    best = -1
+    for i in range(len(vals)):
+        if not allowed[i] or taken[i]:
+            continue
+        if best < 0 or vals[i] > vals[best]:
+            best = i
+    return best
+
+
+def route_token(xt, Wg, bias, k, scale=2.827, norm=True, n_group=1, topk_group=1):
+    """Returns (ids list, weights list) for one token. With n_group > 1 the
+    experts form n_group contiguous groups; a group scores the float32 sum of
+    its two largest keys; only the topk_group best groups' experts compete."""
     E = len(Wg)
     logits = [_dot(xt, Wg[e]) for e in range(E)]
     scores = [_sig(l) for l in logits]
     keys = [_f32(_f32(_sig(_f32(logits[e]))) + _f32(bias[e])) for e in range(E)]
+    gs = E // n_group
+    gscore = []
+    for g in range(n_group):
+        members = keys[g * gs:(g + 1) * gs]
+        first = _best(members, [True] * gs, [False] * gs)
+        rest = [i != first for i in range(gs)]
+        second = _best(members, rest, [False] * gs)
+        gscore.append(members[first] if second < 0 else _f32(members[first] + members[second]))
+    kept_groups = [False] * n_group
+    for _ in range(topk_group):
+        kept_groups[_best(gscore, [True] * n_group, kept_groups)] = True
+    allowed = [kept_groups[e // gs] for e in range(E)]
     taken = [False] * E
     ids = []
     for _ in range(k):
-        best = -1
-        for e in range(E):
-            if taken[e]:
-                continue
-            if best < 0 or keys[e] > keys[best]:
-                best = e
+        best = _best(keys, allowed, taken)
         taken[best] = True
         ids.append(best)
     total = sum(scores[e] for e in ids) if norm else 1.0

@@ -40,8 +40,10 @@ _DECODE_TABLE = np.array([decode_scalar(c) for c in range(256)], dtype=np.float6
 
 
 def decode(codes: np.ndarray) -> np.ndarray:
-    """Vectorised decode of uint8 codes to float64."""
-    return _DECODE_TABLE[np.asarray(codes, dtype=np.uint8)]
+    """Vectorised decode of uint8 codes to float64 (a lookup in the table of
+    decode_scalar's 256 values; the codes are widened to int32 indices first,
+    which numpy gathers several times faster than uint8 ones)."""
+    return np.take(_DECODE_TABLE, np.asarray(codes, dtype=np.uint8).astype(np.int32))
 
 
 def _round_half_even(v: float) -> int:

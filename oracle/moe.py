@@ -34,6 +34,10 @@ Readings taken where the pages are silent (the library follows the same ones):
      nearest-even, saturating), amax = 0 -> s = 1; x is quantised before
      gate/up, the fp32 h = silu(g)*u before down. The router stays fp32 on
      the BF16 x.
+  R19 group-limited routing (n_group > 1): contiguous groups of E / n_group
+     experts, group score = float32 sum of the group's two largest keys, the
+     topk_group best groups kept (ties to the lower group), top-k over their
+     experts only (group_filter). K2 itself has n_group = 1.
 """
 from __future__ import annotations
 
@@ -83,33 +87,81 @@ def topk_by_key(key: np.ndarray, k: int):
     return ids.astype(np.int64), margin
 
 
+def group_filter(keys: np.ndarray, n_group: int, topk_group: int):
+    """Group-limited routing (config fields n_group, topk_group: "Kimi K2
+    Base" raw config table, both 1 for K2; why grouping exists and why K2
+    drops it: "Behind Kimi-K2's Config" §2.4). The pages give no group rule;
+    this library's reading (R19):
+      * the E experts form n_group contiguous groups of E / n_group;
+      * a group's score is the float32 sum of its two largest selection keys
+        (its one key for groups of one expert), decided in float32 as the
+        keys are (R4);
+      * the topk_group groups with the largest scores are kept, ties to the
+        lower group index; every expert of the other groups drops out of the
+        top-k (its key becomes -inf).
+    With n_group = 1 the one group is kept and nothing changes.
+    Returns (keys with the dropped experts at -inf, group margin [T] = the
+    topk_group-th minus the next group score, inf when every group is kept).
+    """
+    keys = np.asarray(keys, np.float32)
+    T, E = keys.shape
+    if n_group < 1 or E % n_group or not 1 <= topk_group <= n_group:
+        raise ValueError("n_group must divide E and 1 <= topk_group <= n_group")
+    gs = E // n_group
+    by_group = -np.sort(-keys.reshape(T, n_group, gs), axis=2)  # each group's keys, descending
+    if gs >= 2:
+        gscore = (by_group[:, :, 0] + by_group[:, :, 1]).astype(np.float32)  # float32 add
+    else:
+        gscore = by_group[:, :, 0]
+    order = np.argsort(-gscore.astype(np.float64), axis=1, kind="stable")  # ties: lower group
+    kept = np.zeros((T, n_group), bool)
+    np.put_along_axis(kept, order[:, :topk_group], True, axis=1)
+    masked = np.where(np.repeat(kept, gs, axis=1), keys, np.float32(-np.inf)).astype(np.float32)
+    if topk_group < n_group:
+        gs_sorted = np.take_along_axis(gscore.astype(np.float64), order, axis=1)
+        gmargin = gs_sorted[:, topk_group - 1] - gs_sorted[:, topk_group]
+    else:
+        gmargin = np.full(T, np.inf)
+    return masked, gmargin
+
+
 @dataclasses.dataclass
 class Routing:
     ids: np.ndarray       # [T, k] int64, slot order = key descending
     weights: np.ndarray   # [T, k] float64, sum = routed_scaling_factor (norm on)
     scores: np.ndarray    # [T, E] float64 unbiased sigmoid scores
-    keys: np.ndarray      # [T, E] float32 selection keys
-    margin: np.ndarray    # [T] float64, k-th minus (k+1)-th key
+    keys: np.ndarray      # [T, E] float32 selection keys (before the group filter)
+    margin: np.ndarray    # [T] float64, k-th minus (k+1)-th key among the kept experts
+    group_margin: Optional[np.ndarray] = None  # [T] topk_group-th minus next group score
 
 
 def route(x, router_weight, bias, k: int, routed_scaling_factor: float = 2.827,
           norm_topk_prob: bool = True, n_group: int = 1, topk_group: int = 1) -> Routing:
-    """Router of the layer: sigmoid scores, noaux_tc biased top-k, normalise, scale."""
-    if n_group != 1 or topk_group != 1:
-        # K2 sets n_group = topk_group = 1 (no grouping): the group filter keeps
-        # every expert. Grouped selection is not part of this layer.
-        raise NotImplementedError("group-limited routing (n_group > 1)")
+    """Router of the layer: sigmoid scores, noaux_tc biased top-k (after the
+    group filter, which keeps every expert when n_group = 1), normalise,
+    scale."""
     logits = router_logits(x, router_weight)
     scores = sigmoid(logits)
     keys = selection_keys(logits, bias)
-    ids, margin = topk_by_key(keys, k)
-    sel = np.take_along_axis(scores, ids, axis=1)
+    masked, gmargin = group_filter(keys, n_group, topk_group)
+    ids, margin = topk_by_key(masked, k)
+    w = routing_weights(scores, ids, routed_scaling_factor, norm_topk_prob)
+    return Routing(ids=ids, weights=w, scores=scores, keys=keys, margin=margin,
+                   group_margin=gmargin)
+
+
+def routing_weights(scores: np.ndarray, ids: np.ndarray, routed_scaling_factor: float = 2.827,
+                    norm_topk_prob: bool = True) -> np.ndarray:
+    """Weights of the chosen experts ids [T, k] from the unbiased scores [T, E]
+    (R2: the bias never enters): normalised over the k chosen scores when
+    norm_topk_prob ("Kimi K2 Base" raw config: norm_topk_prob true), then
+    times routed_scaling_factor (2.827), R5."""
+    sel = np.take_along_axis(np.asarray(scores, np.float64), np.asarray(ids, np.int64), axis=1)
     if norm_topk_prob:
         w = sel / sel.sum(axis=1, keepdims=True)
     else:
         w = sel.copy()
-    w = w * routed_scaling_factor
-    return Routing(ids=ids, weights=w, scores=scores, keys=keys, margin=margin)
+    return w * routed_scaling_factor
 
 
 # --------------------------------------------------------------------------
@@ -185,10 +237,33 @@ def swiglu_expert_fp8(xr: np.ndarray, w_gate: np.ndarray, w_up: np.ndarray,
 ExpertFn = Callable[[int], Dict[str, np.ndarray]]
 
 
-def _as_f64_expert(mats: Dict[str, np.ndarray], fmt: str) -> Dict[str, np.ndarray]:
+def expert_matrices(mats: Dict[str, np.ndarray], fmt: str) -> Dict[str, np.ndarray]:
+    """An expert's gate/up/down as float64 values: BF16 values widened, or FP8
+    codes dequantised with their block scales (R7)."""
     if fmt == "bf16":
         return {n: np.asarray(mats[n], np.float64) for n in ("gate", "up", "down")}
     return {n: weight_dequant(mats[n], mats[n + "_scale"]) for n in ("gate", "up", "down")}
+
+
+def expert_function(fmt: str):
+    """The expert MLP of the weight format: swiglu_expert (BF16) or
+    swiglu_expert_fp8 (activations quantised as R7 states)."""
+    return swiglu_expert if fmt == "bf16" else swiglu_expert_fp8
+
+
+def combine(pair_out: np.ndarray, weights: np.ndarray,
+            shared_out: Optional[np.ndarray] = None) -> np.ndarray:
+    """y[t] = sum_j w[t, j] * pair_out[t, j] + shared_out[t]: the routed
+    outputs weighted and summed in slot order j = 0..k-1, then the shared
+    expert at weight 1, not scaled (R6)."""
+    pair_out = np.asarray(pair_out, np.float64)
+    w = np.asarray(weights, np.float64)
+    y = np.zeros((pair_out.shape[0], pair_out.shape[2]), np.float64)
+    for j in range(pair_out.shape[1]):
+        y += w[:, j:j + 1] * pair_out[:, j]
+    if shared_out is not None:
+        y += shared_out
+    return y
 
 
 def experts_combine(x: np.ndarray, ids: np.ndarray, weights: np.ndarray,
@@ -206,21 +281,18 @@ def experts_combine(x: np.ndarray, ids: np.ndarray, weights: np.ndarray,
     x = np.asarray(x, np.float64)
     toks = np.arange(x.shape[0]) if tokens is None else np.asarray(tokens, np.int64)
     n, k = len(toks), ids.shape[1]
-    ffn = swiglu_expert if fmt == "bf16" else swiglu_expert_fp8
+    ffn = expert_function(fmt)
     pair_out = np.zeros((n, k, x.shape[1]), np.float64)
     sub_ids = np.asarray(ids)[toks]
     for e in np.unique(sub_ids):
         rows, slots = np.nonzero(sub_ids == e)
-        m = _as_f64_expert(get_expert(int(e)), fmt)
+        m = expert_matrices(get_expert(int(e)), fmt)
         pair_out[rows, slots] = ffn(x[toks[rows]], m["gate"], m["up"], m["down"])
-    w = np.asarray(weights, np.float64)[toks]
-    y = np.zeros((n, x.shape[1]), np.float64)
-    for j in range(k):
-        y += w[:, j:j + 1] * pair_out[:, j]
+    shared_out = None
     if get_shared is not None and n_shared_experts > 0:
-        m = _as_f64_expert(get_shared(), fmt)
-        y += ffn(x[toks], m["gate"], m["up"], m["down"])
-    return y
+        m = expert_matrices(get_shared(), fmt)
+        shared_out = ffn(x[toks], m["gate"], m["up"], m["down"])
+    return combine(pair_out, np.asarray(weights, np.float64)[toks], shared_out)
 
 
 def dense_ffn(x: np.ndarray, mats: Dict[str, np.ndarray], fmt: str = "bf16") -> np.ndarray:
@@ -234,18 +306,18 @@ def dense_ffn(x: np.ndarray, mats: Dict[str, np.ndarray], fmt: str = "bf16") -> 
     *_scale block scales, dequantised and with x and h quantised as for the
     experts)."""
     x = np.asarray(x, np.float64)
-    m = _as_f64_expert(mats, fmt)
-    ffn = swiglu_expert if fmt == "bf16" else swiglu_expert_fp8
-    return ffn(x, m["gate"], m["up"], m["down"])
+    m = expert_matrices(mats, fmt)
+    return expert_function(fmt)(x, m["gate"], m["up"], m["down"])
 
 
 def forward(x, router_weight, bias, get_expert: ExpertFn, get_shared, k: int,
             routed_scaling_factor: float = 2.827, norm_topk_prob: bool = True,
             fmt: str = "bf16", n_shared_experts: int = 1,
-            tokens: Optional[Sequence[int]] = None):
+            tokens: Optional[Sequence[int]] = None, n_group: int = 1, topk_group: int = 1):
     """Full layer: route every token, then evaluate the listed tokens (all by
     default). Returns (y float64 [n, d], Routing over all T tokens)."""
-    r = route(x, router_weight, bias, k, routed_scaling_factor, norm_topk_prob)
+    r = route(x, router_weight, bias, k, routed_scaling_factor, norm_topk_prob, n_group,
+              topk_group)
     y = experts_combine(x, r.ids, r.weights, get_expert, get_shared, fmt,
                         n_shared_experts, tokens)
     return y, r

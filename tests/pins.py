@@ -263,7 +263,100 @@ def pin_fp8_exact_grid(orc):
     assert np.array_equal(orc.act_dequant(c2, s2), rows)
 
 
+# ------------------------------------------------------ group-limited routing
+def pin_group_route_vs_brute(orc):
+    """Group-limited routing (n_group > 1) equals the scalar-loop router, for
+    groups of several experts and of one expert each."""
+    for E, ng, tg, k in ((24, 6, 2, 4), (16, 4, 3, 5), (12, 12, 5, 3), (32, 8, 4, 8)):
+        x, Wg, b, _, _ = small_layer(21 + E, T=6, d=32, f=8, E=E, k=k, shared=False)
+        b = b * 10.0  # a wider bias spread: group choices that differ from the plain top-k
+        r = orc.route(x, Wg, b, k, 2.827, True, ng, tg)
+        for t in range(x.shape[0]):
+            ids, w = brute.route_token(x[t], Wg, b, k, 2.827, True, ng, tg)
+            assert list(r.ids[t]) == ids, (E, ng, tg, t, r.ids[t], ids)
+            np.testing.assert_allclose(r.weights[t], w, rtol=1e-12, atol=0)
+
+
+def pin_group_identities(orc):
+    """One group, or every group kept, is the plain top-k: the same ids and
+    weights as a full sort of the keys (ties to the lower index)."""
+    x, Wg, b, _, _ = small_layer(31, T=40, d=24, f=8, E=16, k=4, shared=False)
+    keys = (_sig32(x @ Wg.T) + b.astype(np.float32)).astype(np.float32)
+    plain = np.argsort(-keys.astype(np.float64), axis=1, kind="stable")[:, :4]
+    for ng, tg in ((1, 1), (4, 4), (16, 16)):
+        r = orc.route(x, Wg, b, 4, 2.827, True, ng, tg)
+        assert np.array_equal(r.ids, plain), (ng, tg)
+        assert np.all(np.isinf(r.group_margin))
+
+
+def _sig32(l):
+    l32 = np.asarray(l, np.float64).astype(np.float32).astype(np.float64)
+    return (1.0 / (1.0 + np.exp(-l32))).astype(np.float32)
+
+
+def pin_group_forced(orc):
+    """A +10 bias on every expert of groups 1 and 4 (of 6) with topk_group = 2:
+    those two groups are kept for every token, all chosen experts come from
+    them, their weights are the bias-free normalised scores, and the group
+    margin is about 10."""
+    E, ng, k = 24, 6, 4
+    x, Wg, b, _, _ = small_layer(41, T=30, d=32, f=8, E=E, k=k, shared=False)
+    b = b.copy()
+    forced = np.r_[4:8, 16:20]
+    b[forced] += 10.0
+    r = orc.route(x, Wg, b, k, 2.827, True, ng, 2)
+    assert np.all(np.isin(r.ids, forced))
+    sc = 1.0 / (1.0 + np.exp(-(x @ Wg.T)))
+    sel = np.take_along_axis(sc, r.ids, axis=1)
+    np.testing.assert_allclose(r.weights, 2.827 * sel / sel.sum(1, keepdims=True), rtol=1e-12)
+    assert np.all(r.group_margin > 9.0)
+
+
+def pin_group_invariants(orc):
+    """On many tokens: the chosen experts span at most topk_group groups;
+    every kept group's score (its two largest keys, added in float32) is at
+    least every dropped group's; and the chosen ids are the top-k of the keys
+    of the kept groups' experts."""
+    E, ng, tg, k = 32, 8, 3, 6
+    gs = E // ng
+    x, Wg, b, _, _ = small_layer(51, T=200, d=16, f=8, E=E, k=k, shared=False)
+    b = b * 10.0
+    r = orc.route(x, Wg, b, k, 2.827, True, ng, tg)
+    keys = r.keys.astype(np.float32)
+    for t in range(x.shape[0]):
+        g_of = r.ids[t] // gs
+        assert len(set(g_of.tolist())) <= tg
+        top2 = []
+        for g in range(ng):
+            kk = sorted(keys[t, g * gs:(g + 1) * gs].tolist(), reverse=True)
+            top2.append(float(np.float32(kk[0]) + np.float32(kk[1])))
+        kept = sorted(range(ng), key=lambda g: (-top2[g], g))[:tg]
+        assert set(g_of.tolist()) <= set(kept)
+        assert min(top2[g] for g in kept) >= max(top2[g] for g in range(ng) if g not in kept)
+        cand = [e for e in range(E) if e // gs in kept]
+        want = sorted(cand, key=lambda e: (-float(keys[t, e]), e))[:k]
+        assert list(r.ids[t]) == want
+
+
+def pin_group_tie_rule(orc):
+    """Equal group scores keep the lower group: with a zero router every score
+    is 1/2, so the keys are 1/2 + bias; groups 1 and 3 (of 4) get the same two
+    largest biases, and topk_group = 1 must keep group 1."""
+    E, ng, d = 16, 4, 8
+    x = np.ones((3, d))
+    Wg = np.zeros((E, d))
+    b = np.zeros(E)
+    b[[5, 6]] = [0.25, 0.125]     # group 1
+    b[[13, 15]] = [0.125, 0.25]   # group 3: the same two values
+    b[[0, 8]] = [0.2, 0.2]        # groups 0 and 2: lower sums
+    r = orc.route(x, Wg, b, 2, 2.827, True, ng, 1)
+    assert np.all(r.ids == np.array([5, 6]))
+    assert np.all(r.group_margin == 0.0)
+
+
 ALL_PINS = [pin_route_vs_brute, pin_layer_vs_brute_bf16, pin_layer_vs_brute_fp8,
             pin_weights_sum, pin_bias_selects_only, pin_k_equals_E,
             pin_identical_experts_closed_form, pin_textbook_values, pin_printed_counts,
-            pin_act_quant, pin_fp8_exact_grid, pin_dense_ffn_vs_brute]
+            pin_act_quant, pin_fp8_exact_grid, pin_dense_ffn_vs_brute,
+            pin_group_route_vs_brute, pin_group_identities, pin_group_forced,
+            pin_group_invariants, pin_group_tie_rule]

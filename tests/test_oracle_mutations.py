@@ -11,18 +11,17 @@ from tests import pins
 
 def _bad_route_weights_from_keys(x, router_weight, bias, k, routed_scaling_factor=2.827,
                                  norm_topk_prob=True, n_group=1, topk_group=1):
-    logits = orc.router_logits(x, router_weight)
-    keys = orc.selection_keys(logits, bias)
-    ids, margin = orc.topk_by_key(keys, k)
-    sel = np.take_along_axis(keys.astype(np.float64), ids, axis=1)  # biased keys as weights
-    w = sel / sel.sum(axis=1, keepdims=True) * routed_scaling_factor
-    return orc.Routing(ids, w, orc.sigmoid(logits), keys, margin)
+    r = _GOOD_ROUTE(x, router_weight, bias, k, routed_scaling_factor, norm_topk_prob, n_group,
+                    topk_group)
+    sel = np.take_along_axis(r.keys.astype(np.float64), r.ids, axis=1)  # biased keys as weights
+    r.weights = sel / sel.sum(axis=1, keepdims=True) * routed_scaling_factor
+    return r
 
 
 def _bad_route_no_norm(x, router_weight, bias, k, routed_scaling_factor=2.827,
                        norm_topk_prob=True, n_group=1, topk_group=1):
-    r = _GOOD_ROUTE(x, router_weight, bias, k, routed_scaling_factor, False)
-    return r
+    return _GOOD_ROUTE(x, router_weight, bias, k, routed_scaling_factor, False, n_group,
+                       topk_group)
 
 
 def _bad_topk_ascending(key, k):
@@ -79,6 +78,51 @@ def _shared_scaled_combine(x, ids, weights, get_expert, get_shared, fmt="bf16",
 
 
 _GOOD_COMBINE = orc.experts_combine
+_GOOD_GROUP_FILTER = orc.group_filter
+_GOOD_COMBINE_SUM = orc.combine
+
+
+def _bad_group_score_max(keys, n_group, topk_group):
+    # planted: a group scores its largest key only
+    keys = np.asarray(keys, np.float32)
+    T, E = keys.shape
+    gs = E // n_group
+    g = keys.reshape(T, n_group, gs).max(axis=2)
+    order = np.argsort(-g.astype(np.float64), axis=1, kind="stable")
+    kept = np.zeros((T, n_group), bool)
+    np.put_along_axis(kept, order[:, :topk_group], True, axis=1)
+    masked = np.where(np.repeat(kept, gs, axis=1), keys, np.float32(-np.inf)).astype(np.float32)
+    return masked, np.full(T, np.inf)
+
+
+def _bad_group_strided(keys, n_group, topk_group):
+    # planted: group g holds the experts e with e % n_group == g
+    keys = np.asarray(keys, np.float32)
+    T, E = keys.shape
+    perm = np.argsort(np.arange(E) % n_group, kind="stable")
+    inv = np.argsort(perm)
+    masked, gm = _GOOD_GROUP_FILTER(keys[:, perm], n_group, topk_group)
+    return masked[:, inv], gm
+
+
+def _bad_group_ties_high(keys, n_group, topk_group):
+    # planted: equal group scores keep the higher group
+    keys = np.asarray(keys, np.float32)
+    T, E = keys.shape
+    rev = np.arange(E).reshape(n_group, E // n_group)[::-1].ravel()
+    masked, gm = _GOOD_GROUP_FILTER(keys[:, rev], n_group, topk_group)
+    return masked[:, np.argsort(rev)], gm
+
+
+def _bad_routing_weights_unnormalised(scores, ids, routed_scaling_factor=2.827,
+                                      norm_topk_prob=True):
+    sel = np.take_along_axis(np.asarray(scores, np.float64), np.asarray(ids, np.int64), axis=1)
+    return sel * routed_scaling_factor
+
+
+def _bad_combine_shared_scaled(pair_out, weights, shared_out=None):
+    return _GOOD_COMBINE_SUM(pair_out, weights,
+                             None if shared_out is None else 2.827 * shared_out)
 
 MUTATIONS = {
     "weights_from_biased_keys": ("route", _bad_route_weights_from_keys),
@@ -91,6 +135,11 @@ MUTATIONS = {
     "act_quant_wrong_scale": ("act_quant", _bad_act_quant_scale),
     "weight_scale_misindexed": ("weight_dequant", _bad_weight_dequant_transposed_blocks),
     "expert_params_two_mats": ("expert_params", _bad_expert_params),
+    "group_score_max_key": ("group_filter", _bad_group_score_max),
+    "group_strided": ("group_filter", _bad_group_strided),
+    "group_ties_to_higher": ("group_filter", _bad_group_ties_high),
+    "routing_weights_unnormalised": ("routing_weights", _bad_routing_weights_unnormalised),
+    "combine_shared_scaled": ("combine", _bad_combine_shared_scaled),
 }
 
 
