@@ -6,7 +6,8 @@
  *   - Router: logits = x . W_g^T over n_routed_experts = 384 experts of
  *     hidden_size = 7168 inputs, scoring_func = sigmoid,
  *     topk_method = noaux_tc (an additive e_score_correction_bias is used to
- *     choose experts only), n_group = topk_group = 1 (no group filter),
+ *     choose experts only), n_group = topk_group = 1 (no group filter;
+ *     other values select group-limited routing, see moe_config_t),
  *     num_experts_per_tok = 8, norm_topk_prob = true (the 8 chosen unbiased
  *     scores are normalised to sum 1), routed_scaling_factor = 2.827.
  *     Source: "Kimi K2 Base" and "Kimi K2 0905" model cards, raw config.json
@@ -86,8 +87,17 @@ typedef struct {
    * first_k_dense_replace 1, intermediate_size 18432) is f = 2048,
    * n_shared_experts = 9. The router and routed-expert weights are then
    * ignored (may be NULL). */
-  int32_t n_group;                /* must be 1 (K2) */
-  int32_t topk_group;             /* must be 1 (K2) */
+  /* Group-limited routing (1, 1 for K2: no groups). With n_group > 1 the
+   * experts form n_group contiguous groups of n_routed_experts / n_group; a
+   * group's score is the fp32 sum of its two largest selection keys (its one
+   * key for groups of one expert); only the experts of the topk_group groups
+   * with the largest scores (ties to the lower group) take part in the top-k.
+   * The pages give the two fields and why K2 sets them to 1 ("Behind
+   * Kimi-K2's Config" §2.4), not the group rule: this rule is the library's
+   * reading. Needs n_group <= 32 dividing n_routed_experts, 1 <= topk_group
+   * <= n_group, and num_experts_per_tok <= topk_group * group size. */
+  int32_t n_group;
+  int32_t topk_group;
   int32_t norm_topk_prob;         /* 1 (K2): normalise the k scores; 0: do not */
   float routed_scaling_factor;    /* 2.827 for K2 */
   int32_t scoring_func;           /* MOE_SCORING_SIGMOID */
@@ -121,6 +131,13 @@ typedef struct {
 
 /* moe_forward_opts_t.flags */
 #define MOE_FLAG_SYNC_CHECK 0x1u /* synchronise the stream and read the device status word */
+/* Test hook for the failure path: the gate/up GEMM's MMA issuer waits on a
+ * barrier that nothing signals. The wait runs out after wait_limit_ns (below),
+ * sets MOE_DEVICE_WAIT_TIMEOUT, and every CTA winds down (waits for its own
+ * loads in flight, frees its tensor memory, returns); the rest of the
+ * forward runs on, so y holds no meaningful values. Nothing faults or hangs:
+ * it is the path a real timeout takes. */
+#define MOE_FLAG_TEST_STALL 0x2u
 
 typedef struct {
   int32_t* topk_ids_out;          /* optional device [T, k]: chosen experts, key-descending */
@@ -131,6 +148,19 @@ typedef struct {
                                      status word gets MOE_DEVICE_BAD_EXPERT_ID */
   float* router_logits_out;       /* optional device [T, E]: the router logits x . W_g^T */
   uint32_t flags;                 /* MOE_FLAG_* */
+  uint32_t reserved;              /* must be 0 */
+  /* optional device [E + 1]: row offsets of the routed experts in the grouped
+   * GEMMs' row order. Expert e's rows are [offsets[e], offsets[e+1]), in
+   * ascending token order; offsets[0] = 0, offsets[E] = T * k. */
+  int32_t* expert_offsets_out;
+  /* optional device [T, k]: the row of each (token, slot) pair in that order
+   * (a bijection onto [0, T * k)). */
+  int32_t* pair_rows_out;
+  /* Time limit of each pipeline wait in the GEMM kernels, in ns; 0 = the
+   * default of 2 s. A wait that runs out sets MOE_DEVICE_WAIT_TIMEOUT. The
+   * wind-down after it (waiting for loads and MMAs already in flight) keeps
+   * the default limit. */
+  uint64_t wait_limit_ns;
 } moe_forward_opts_t;
 
 /* Device status word bits (moe_get_device_status) */
@@ -144,7 +174,7 @@ moe_status_t moe_config_init_k2(moe_config_t* cfg);
 
 /* Validate cfg, select `device`, allocate the handle's weight buffers and a
  * workspace for up to cfg->max_tokens tokens. Unsupported values
- * (n_group != 1, other scoring or top-k methods, sizes not multiples of 128)
+ * (n_group > 32, other scoring or top-k methods, sizes not multiples of 128)
  * return MOE_ERR_UNSUPPORTED. Synchronous. */
 moe_status_t moe_create(const moe_config_t* cfg, int device, moe_handle_t** out);
 
@@ -227,11 +257,15 @@ int64_t moe_launch_count(const moe_handle_t* h);
  * The pages have no counterpart of this call; it exists for callers that
  * cannot call cudaMalloc: engines that hand nearly all GPU memory to their
  * own pool at start-up, and latency-critical steps that cannot afford the
- * device synchronisation cudaMalloc may cause. It computes what moe_forward
- * computes for routing (the same kernels): for T tokens, the
- * num_experts_per_tok experts with the largest sigmoid score + bias, key
- * descending, and their weights (unbiased scores, normalised when
- * norm_topk_prob = 1, times routed_scaling_factor).
+ * device synchronisation cudaMalloc may cause. It computes the routing that
+ * moe_forward computes: for T tokens, the num_experts_per_tok experts with
+ * the largest sigmoid score + bias, key descending, and their weights
+ * (unbiased scores, normalised when norm_topk_prob = 1, times
+ * routed_scaling_factor). Its logits always come from the split-K fp32
+ * CUDA-core kernel, which moe_forward uses for 8 < T < 512 only (a GEMV for
+ * T <= 8, the tensor-core router for T >= 512); those sum the logits in
+ * another order, so a token whose k-th and (k+1)-th keys are within about
+ * 1e-5 may choose differently, and weights may differ in the last bits.
  *
  *   x              device BF16 [T, hidden_size], 16-byte aligned
  *   router_weight  device fp32 [n_routed_experts, hidden_size], 16-byte aligned
@@ -250,7 +284,10 @@ int64_t moe_launch_count(const moe_handle_t* h);
  * array: calls whose GPU work can overlap (unordered streams, several host
  * threads) race and must not be made. hidden_size must be a multiple of 32,
  * n_routed_experts <= 512, num_experts_per_tok <= 32 (else
- * MOE_ERR_UNSUPPORTED). */
+ * MOE_ERR_UNSUPPORTED). The call does not wait for the GPU, so it reports
+ * only what the host checks: problems its kernels find are not reported
+ * (NaN keys, for one, silently get the smallest expert ids not yet
+ * taken). */
 moe_status_t moe_router_topk_noalloc(const void* x, int64_t T, const float* router_weight,
                                      const float* e_score_correction_bias, int32_t hidden_size,
                                      int32_t n_routed_experts, int32_t num_experts_per_tok,

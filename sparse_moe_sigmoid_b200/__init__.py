@@ -35,6 +35,7 @@ MOE_SCORING_SIGMOID = 0
 MOE_TOPK_NOAUX_TC = 0
 MOE_ACTIVATION_DYNAMIC = 0
 MOE_FLAG_SYNC_CHECK = 0x1
+MOE_FLAG_TEST_STALL = 0x2
 MOE_DEVICE_WAIT_TIMEOUT = 0x1
 MOE_DEVICE_BAD_EXPERT_ID = 0x2
 MOE_NUM_PHASES = 7
@@ -63,7 +64,9 @@ class moe_weights_t(ctypes.Structure):
 class moe_forward_opts_t(ctypes.Structure):
     _fields_ = [("topk_ids_out", ctypes.c_void_p), ("topk_weights_out", ctypes.c_void_p),
                 ("forced_topk_ids", ctypes.c_void_p), ("router_logits_out", ctypes.c_void_p),
-                ("flags", ctypes.c_uint32)]
+                ("flags", ctypes.c_uint32), ("reserved", ctypes.c_uint32),
+                ("expert_offsets_out", ctypes.c_void_p), ("pair_rows_out", ctypes.c_void_p),
+                ("wait_limit_ns", ctypes.c_uint64)]
 
 
 _H = ctypes.c_void_p
@@ -168,21 +171,28 @@ def moe_load_weights(h, router_weight, e_score_correction_bias, gate_proj, up_pr
     _check(_lib.moe_load_weights(h, ctypes.byref(w), _stream(stream)), "moe_load_weights", h)
 
 
-def _opts(topk_ids_out, topk_weights_out, forced_topk_ids, router_logits_out, flags):
+def _opts(topk_ids_out=None, topk_weights_out=None, forced_topk_ids=None,
+          router_logits_out=None, flags=0, expert_offsets_out=None, pair_rows_out=None,
+          wait_limit_ns=0):
     if (topk_ids_out is None and topk_weights_out is None and forced_topk_ids is None
-            and router_logits_out is None and not flags):
+            and router_logits_out is None and not flags and expert_offsets_out is None
+            and pair_rows_out is None and not wait_limit_ns):
         return None
-    return ctypes.byref(moe_forward_opts_t(_ptr(topk_ids_out), _ptr(topk_weights_out),
-                                           _ptr(forced_topk_ids), _ptr(router_logits_out), flags))
+    return ctypes.byref(moe_forward_opts_t(
+        _ptr(topk_ids_out), _ptr(topk_weights_out), _ptr(forced_topk_ids),
+        _ptr(router_logits_out), flags, 0, _ptr(expert_offsets_out), _ptr(pair_rows_out),
+        wait_limit_ns))
 
 
 def moe_forward(h, x, y, T: Optional[int] = None, topk_ids_out=None, topk_weights_out=None,
-                forced_topk_ids=None, router_logits_out=None, flags: int = 0, stream=None):
+                forced_topk_ids=None, router_logits_out=None, flags: int = 0, stream=None,
+                expert_offsets_out=None, pair_rows_out=None, wait_limit_ns: int = 0):
     """y = MoE(x); x and y are BF16 [T, hidden] device tensors."""
     T = x.shape[0] if T is None else T
     st = _lib.moe_forward(h, _ptr(x), T, _ptr(y),
                           _opts(topk_ids_out, topk_weights_out, forced_topk_ids,
-                                router_logits_out, flags),
+                                router_logits_out, flags, expert_offsets_out, pair_rows_out,
+                                wait_limit_ns),
                           _stream(stream))
     _check(st, "moe_forward", h)
 
@@ -191,7 +201,7 @@ def moe_forward_host(h, x_host, y_host, T: Optional[int] = None, flags: int = 0,
     """The same from host (CPU, ideally pinned) BF16 tensors; synchronises."""
     T = x_host.shape[0] if T is None else T
     st = _lib.moe_forward_host(h, _ptr(x_host), T, _ptr(y_host),
-                               _opts(None, None, None, None, flags), _stream(stream))
+                               _opts(flags=flags), _stream(stream))
     _check(st, "moe_forward_host", h)
 
 
@@ -201,7 +211,7 @@ def moe_forward_host_async(h, x_host, y_host, T: Optional[int] = None, flags: in
     y_host unread, and both alive, until moe_host_wait(h) returns."""
     T = x_host.shape[0] if T is None else T
     st = _lib.moe_forward_host_async(h, _ptr(x_host), T, _ptr(y_host),
-                                     _opts(None, None, None, None, flags), _stream(stream))
+                                     _opts(flags=flags), _stream(stream))
     _check(st, "moe_forward_host_async", h)
 
 

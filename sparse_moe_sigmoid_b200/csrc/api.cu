@@ -131,8 +131,16 @@ moe_status_t validate(const moe_config_t* c, std::string* why) {
   if (c->n_routed_experts > smoe::kMaxExperts) return unsup("n_routed_experts > 512");
   if (c->num_experts_per_tok > smoe::kMaxTopK) return unsup("num_experts_per_tok > 32");
   if (c->n_shared_experts > 16) return unsup("n_shared_experts > 16");
-  if (c->n_group != 1 || c->topk_group != 1)
-    return unsup("group-limited routing (n_group/topk_group != 1) is not implemented");
+  if (c->n_group < 1 || c->topk_group < 1 || c->topk_group > c->n_group)
+    return bad("need 1 <= topk_group <= n_group");
+  if (c->n_routed_experts == 0 && (c->n_group != 1 || c->topk_group != 1))
+    return bad("without routed experts: n_group = topk_group = 1");
+  if (c->n_group > 32) return unsup("n_group > 32");
+  if (c->n_routed_experts > 0 && c->n_routed_experts % c->n_group)
+    return bad("n_group must divide n_routed_experts");
+  if (c->n_routed_experts > 0 &&
+      c->num_experts_per_tok > c->topk_group * (c->n_routed_experts / c->n_group))
+    return bad("num_experts_per_tok exceeds the experts of topk_group groups");
   if (c->scoring_func != MOE_SCORING_SIGMOID) return unsup("scoring_func must be sigmoid");
   if (c->topk_method != MOE_TOPK_NOAUX_TC) return unsup("topk_method must be noaux_tc");
   if (c->norm_topk_prob != 0 && c->norm_topk_prob != 1) return bad("norm_topk_prob is 0 or 1");
@@ -471,6 +479,8 @@ moe_status_t moe_forward(moe_handle_t* h, const void* x, int64_t T, void* y,
     return fail(h, MOE_ERR_INVALID_ARG, "x and y overlap");
   if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 15)
     return fail(h, MOE_ERR_INVALID_ARG, "x and y must be 16-byte aligned");
+  if (opts && (opts->reserved != 0 || (opts->flags & ~(MOE_FLAG_SYNC_CHECK | MOE_FLAG_TEST_STALL))))
+    return fail(h, MOE_ERR_INVALID_ARG, "unknown option flags, or reserved != 0");
   DeviceGuard guard(h->device);
   if (!guard.ok) return fail(h, MOE_ERR_CUDA, "cudaSetDevice failed");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -499,6 +509,15 @@ moe_status_t launch_forward(moe_handle* h, const void* x, int64_t T, void* y,
                      : T <= smoe::kRouterGemvMaxT ? 1  // the GEMV router: one slice
                                                   : smoe::router_splits(dm, T, h->num_sms);
   const int32_t* forced = opts ? opts->forced_topk_ids : nullptr;
+  h->fwd_wait_ns = opts ? opts->wait_limit_ns : 0;
+  h->fwd_stall = opts && (opts->flags & MOE_FLAG_TEST_STALL);
+  struct Reset {  // the next forward starts from the defaults again
+    moe_handle* h;
+    ~Reset() {
+      h->fwd_wait_ns = 0;
+      h->fwd_stall = false;
+    }
+  } reset{h};
 
   mark(0);
   CUDA_TRY(h, cudaMemsetAsync(h->ws.sched, 0, h->ws.zero_bytes, s), "clear counts");
@@ -525,6 +544,14 @@ moe_status_t launch_forward(moe_handle* h, const void* x, int64_t T, void* y,
   CUDA_TRY(h, smoe::launch_route_scan(h, Ti, p1, p2, s), "route scan launch");
   mark(3);
   CUDA_TRY(h, smoe::launch_dispatch(h, x, Ti, s), "dispatch launch");
+  if (opts && opts->expert_offsets_out && dm.E > 0)
+    CUDA_TRY(h, cudaMemcpyAsync(opts->expert_offsets_out, h->ws.offsets, (dm.E + 1) * 4,
+                                cudaMemcpyDeviceToDevice, s),
+             "offsets copy");
+  if (opts && opts->pair_rows_out && dm.E > 0)
+    CUDA_TRY(h, cudaMemcpyAsync(opts->pair_rows_out, h->ws.pair_row, T * dm.k * 4,
+                                cudaMemcpyDeviceToDevice, s),
+             "pair rows copy");
   mark(4);
   if (dm.fp8) {
     CUDA_TRY(h, smoe::launch_gemm_fp8(h, true, p1, s), "gate/up GEMM launch");

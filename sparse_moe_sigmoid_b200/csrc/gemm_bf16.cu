@@ -54,7 +54,7 @@ struct Bf16Cfg {
   static constexpr int kAccCols = NA * BN;
   static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
   static constexpr int kTmemCols = pow2_at_least(kAccBufs * kAccCols, 32);
-  static constexpr int kSmem = kStages * kStage + 1024 + 256;
+  static constexpr int kSmem = kStages * kStage + 1024 + 256;  // + barriers and flags
   static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(kTmemCols <= 512, "TMEM holds 512 columns");
   static_assert(kStages >= 2, "need at least two stages");
@@ -80,7 +80,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* stallbar = drain + 1;  // test hook: never signalled
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stallbar + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* consumed = tmem_slot + 2;
   volatile uint32_t* issued = tmem_slot + 3;
@@ -98,6 +99,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&tempty[a], 4);
     }
     mbar_init(drain, 1);
+    mbar_init(stallbar, 1);
     *abort_flag = 0;
     *consumed = 0;
     *issued = 0;
@@ -118,6 +120,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total_units = total_units_of(args, BN);
+  const uint64_t lim = wait_limit(args);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -128,7 +131,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int kb = 0; kb < args.k_blocks; ++kb, ++it) {
           const int s = it % C::kStages;
           const uint32_t ph = (it / C::kStages) & 1u;
-          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim)) {
             ok = false;
             break;
           }
@@ -149,13 +152,14 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       uint32_t it = 0;
-      bool ok = true;
+      // the test hook's wait on a barrier nothing signals runs out after lim
+      bool ok = !args.stall || mbar_wait(stallbar, 0, abort_flag, lim);
       int i = 0;
       for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++i) {
         const Unit un = decode_unit(u, args, BN);
         const int acc = i % C::kAccBufs;
         const int use = i / C::kAccBufs;
-        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag)) {
+        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag, lim)) {
           ok = false;
           break;
         }
@@ -166,7 +170,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int kb = 0; kb < args.k_blocks; ++kb, ++it) {
           const int s = it % C::kStages;
           const uint32_t ph = (it / C::kStages) & 1u;
-          if (!mbar_wait(&full[s], ph, abort_flag)) {
+          if (!mbar_wait(&full[s], ph, abort_flag, lim)) {
             ok = false;
             break;
           }
@@ -203,7 +207,7 @@ __global__ void __launch_bounds__(192, 1)
       const Unit un = decode_unit(u, args, BN);
       const int acc = i % C::kAccBufs;
       const int use = i / C::kAccBufs;
-      if (!mbar_wait(&tfull[acc], use & 1, abort_flag)) {
+      if (!mbar_wait(&tfull[acc], use & 1, abort_flag, lim)) {
         if (lane == 0) {
           *abort_flag = 1;
           atomicOr(args.status, MOE_DEVICE_WAIT_TIMEOUT);
@@ -282,6 +286,8 @@ cudaError_t launch_gemm_bf16(moe_handle* h, bool gated, const GemmPlan& p, cudaS
   a.k_blocks = p.k_blocks;
   a.bn = p.bn;
   a.status = h->ws.status;
+  a.wait_ns = h->fwd_wait_ns;
+  a.stall = gated && h->fwd_stall ? 1 : 0;
   a.b_k = gated ? dm.d : dm.f;
   a.m_valid = gated ? dm.f : dm.d;
   const int bi = bn_index(p.bn);

@@ -91,8 +91,11 @@ struct Pair2Cfg {
   static constexpr int kChunksPerWarp = BN / 32;
 };
 
+// silu(g) * u with IEEE expf and division, the same arithmetic as the 1-SM
+// and FP8 kernels, so a token's h does not depend on which kernel its batch
+// size selects.
 __device__ __forceinline__ float silu_mul(float g, float u) {
-  return __fdividef(g, 1.f + __expf(-g)) * u;
+  return g / (1.f + expf(-g)) * u;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -114,7 +117,8 @@ __global__ void __maxnreg__(kPairRegs)
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint64_t* uq_full = drain + 1;           // [kUnitRing] a unit index was published
+  uint64_t* stallbar = drain + 1;          // test hook: never signalled
+  uint64_t* uq_full = stallbar + 1;        // [kUnitRing] a unit index was published
   uint64_t* uq_empty = uq_full + kUnitRing;  // [kUnitRing] (even CTA) every reader has it
   int32_t* uq = reinterpret_cast<int32_t*>(uq_empty + kUnitRing);  // [kUnitRing]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(uq + kUnitRing);
@@ -139,6 +143,7 @@ __global__ void __maxnreg__(kPairRegs)
       mbar_init(&tempty[a], 2 * kPairEpiWarps);  // the epilogue warps of both CTAs
     }
     mbar_init(drain, 1);
+    mbar_init(stallbar, 1);
     for (int j = 0; j < kUnitRing; ++j) {
       mbar_init(&uq_full[j], 1);
       mbar_init(&uq_empty[j], kUnitReaders);
@@ -164,6 +169,7 @@ __global__ void __maxnreg__(kPairRegs)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total_units = total_units_of(args, BN);
+  const uint64_t lim = wait_limit(args);
   // j-th unit index of this pair (every reader; false: a wait gave up)
   auto read_unit = [&](uint32_t j, int* u) -> bool {
     if (!dynamic) {
@@ -172,8 +178,8 @@ __global__ void __maxnreg__(kPairRegs)
     }
     const int slot = static_cast<int>(j % kUnitRing);
     const uint32_t ph = (j / kUnitRing) & 1u;
-    const bool ok = rank == 0 ? mbar_wait(&uq_full[slot], ph, abort_flag)
-                              : mbar_wait_cluster(&uq_full[slot], ph, abort_flag);
+    const bool ok = rank == 0 ? mbar_wait(&uq_full[slot], ph, abort_flag, lim)
+                              : mbar_wait_cluster(&uq_full[slot], ph, abort_flag, lim);
     if (!ok) return false;
     *u = uq[slot];
     return true;
@@ -197,7 +203,7 @@ __global__ void __maxnreg__(kPairRegs)
         if (dynamic && rank == 0) {
           // publish the next unit to both CTAs
           const int slot = static_cast<int>(j % kUnitRing);
-          if (!mbar_wait_cluster(&uq_empty[slot], ((j / kUnitRing) & 1u) ^ 1u, abort_flag)) {
+          if (!mbar_wait_cluster(&uq_empty[slot], ((j / kUnitRing) & 1u) ^ 1u, abort_flag, lim)) {
             ok = false;
             break;
           }
@@ -224,7 +230,7 @@ __global__ void __maxnreg__(kPairRegs)
         for (int ks = 0; ks < args.k_blocks / C::kKSub; ++ks, ++it) {
           const int s = it % C::kStages;
           const uint32_t ph = (it / C::kStages) & 1u;
-          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim)) {
             ok = false;
             break;
           }
@@ -249,7 +255,8 @@ __global__ void __maxnreg__(kPairRegs)
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       uint32_t it = 0;
-      bool ok = true;
+      // the test hook's wait on a barrier nothing signals runs out after lim
+      bool ok = !args.stall || mbar_wait(stallbar, 0, abort_flag, lim);
       for (uint32_t i = 0; ok; ++i) {
         int u;
         if (!read_unit(i, &u)) {
@@ -261,7 +268,7 @@ __global__ void __maxnreg__(kPairRegs)
         const Unit un = decode_unit(u, args, BN);
         const int acc = i % C::kAccBufs;
         const int use = i / C::kAccBufs;
-        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag)) {
+        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag, lim)) {
           ok = false;
           break;
         }
@@ -272,7 +279,7 @@ __global__ void __maxnreg__(kPairRegs)
         for (int ks = 0; ks < args.k_blocks / C::kKSub; ++ks, ++it) {
           const int s = it % C::kStages;
           const uint32_t ph = (it / C::kStages) & 1u;
-          if (!mbar_wait(&full[s], ph, abort_flag)) {
+          if (!mbar_wait(&full[s], ph, abort_flag, lim)) {
             ok = false;
             break;
           }
@@ -321,7 +328,7 @@ __global__ void __maxnreg__(kPairRegs)
       const Unit un = decode_unit(u, args, BN);
       const int acc = i % C::kAccBufs;
       const int use = i / C::kAccBufs;
-      if (!mbar_wait(&tfull[acc], use & 1, abort_flag)) {
+      if (!mbar_wait(&tfull[acc], use & 1, abort_flag, lim)) {
         if (lane == 0) {
           *abort_flag = 1;
           atomicOr(args.status, MOE_DEVICE_WAIT_TIMEOUT);
@@ -457,6 +464,8 @@ cudaError_t launch_gemm_bf16_pair(moe_handle* h, bool gated, const GemmPlan& p, 
   a.k_blocks = p.k_blocks;
   a.bn = p.bn;
   a.status = h->ws.status;
+  a.wait_ns = h->fwd_wait_ns;
+  a.stall = gated && h->fwd_stall ? 1 : 0;
   a.b_k = gated ? dm.d : dm.f;
   a.m_valid = gated ? dm.f : dm.d;
   a.sched = gated ? h->ws.sched : nullptr;  // dynamic units for gate/up only

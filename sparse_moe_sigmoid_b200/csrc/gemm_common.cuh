@@ -13,6 +13,8 @@
 
 #include <stdint.h>
 
+#include "sm100.cuh"
+
 namespace smoe {
 
 struct Unit {
@@ -48,7 +50,14 @@ struct GemmArgs {
                              // partial result at out + s * split_stride elements
   size_t split_stride;
   int out_bf16;               // promoted GEMM, plain mode: outputs stored BF16 (else fp32)
+  uint64_t wait_ns;           // limit of each pipeline wait (the wind-down keeps the default)
+  int stall;                  // test hook: the MMA issuer waits on a barrier nothing signals
 };
+
+// Limit of a pipeline wait: the caller's, or the default.
+__device__ __forceinline__ uint64_t wait_limit(const GemmArgs& a) {
+  return a.wait_ns ? a.wait_ns : sm100::kTimeoutNs;
+}
 
 __device__ __forceinline__ int total_units_of(const GemmArgs& a, int BN) {
   return a.unit_base ? __ldg(a.unit_base + a.G)

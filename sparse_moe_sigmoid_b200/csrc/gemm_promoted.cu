@@ -156,7 +156,8 @@ __global__ void __maxnreg__(prom_regs<NPG>())
   uint64_t* pempty = pfull + 4;
   uint64_t* drain = pempty + 4;
   uint64_t* grp = drain + 1;  // the promotion threads' own barrier (bounded waits)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(grp + 1);
+  uint64_t* stallbar = grp + 1;  // test hook: never signalled
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stallbar + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* consumed = tmem_slot + 2;
   volatile uint32_t* issued = tmem_slot + 3;
@@ -176,6 +177,7 @@ __global__ void __maxnreg__(prom_regs<NPG>())
     }
     mbar_init(drain, 1);
     mbar_init(grp, 128 * NPG);
+    mbar_init(stallbar, 1);
     *abort_flag = 0;
     *consumed = 0;
     *issued = 0;
@@ -196,6 +198,7 @@ __global__ void __maxnreg__(prom_regs<NPG>())
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total_units = total_units_of(args, BN);
+  const uint64_t lim = wait_limit(args);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -206,7 +209,7 @@ __global__ void __maxnreg__(prom_regs<NPG>())
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1u;
-          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim)) {
             ok = false;
             break;
           }
@@ -229,7 +232,8 @@ __global__ void __maxnreg__(prom_regs<NPG>())
     if (lane == 0) {
       uint32_t it = 0;   // stages consumed so far
       uint32_t pit = 0;  // promotions handed over so far (the partial-buffer sequence)
-      bool ok = true;
+      // the test hook's wait on a barrier nothing signals runs out after lim
+      bool ok = !args.stall || mbar_wait(stallbar, 0, abort_flag, lim);
       for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
         const Unit un = decode_unit(u, args, BN);
         const uint32_t n = static_cast<uint32_t>(((un.nvalid + 15) / 16) * 16);
@@ -240,8 +244,8 @@ __global__ void __maxnreg__(prom_regs<NPG>())
           const int pb = pit % C::kPBufs;
           const int sub = kb % KPP;
           if ((sub == 0 &&
-               !mbar_wait(&pempty[pb], ((pit / C::kPBufs) & 1u) ^ 1u, abort_flag)) ||
-              !mbar_wait(&full[s], ph, abort_flag)) {
+               !mbar_wait(&pempty[pb], ((pit / C::kPBufs) & 1u) ^ 1u, abort_flag, lim)) ||
+              !mbar_wait(&full[s], ph, abort_flag, lim)) {
             ok = false;
             break;
           }
@@ -284,7 +288,7 @@ __global__ void __maxnreg__(prom_regs<NPG>())
     bool ok = true;
     auto group_sync = [&]() {
       mbar_arrive(grp);
-      const bool r = mbar_wait(grp, gph, abort_flag);
+      const bool r = mbar_wait(grp, gph, abort_flag, lim);
       gph ^= 1u;
       return r;
     };
@@ -325,7 +329,7 @@ __global__ void __maxnreg__(prom_regs<NPG>())
       const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
       for (int pg = 0; pg < NP; ++pg, ++pit) {
         const int pb = pit % C::kPBufs;
-        if (!mbar_wait(&pfull[pb], (pit / C::kPBufs) & 1u, abort_flag)) {
+        if (!mbar_wait(&pfull[pb], (pit / C::kPBufs) & 1u, abort_flag, lim)) {
           ok = false;
           break;
         }
@@ -508,6 +512,8 @@ cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaSt
   a.k_blocks = p.k_blocks;
   a.bn = p.bn;
   a.status = h->ws.status;
+  a.wait_ns = h->fwd_wait_ns;
+  a.stall = gated && h->fwd_stall ? 1 : 0;
   a.b_k = gated ? dm.d : dm.f;
   a.m_valid = gated ? dm.f : dm.d;
   const int bi = bn_index(p.bn);

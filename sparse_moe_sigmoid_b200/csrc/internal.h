@@ -87,6 +87,10 @@ struct moe_handle {
   CUtensorMap tm_xp[16], tm_h[16];
   int router_max_splits = 1;
   int64_t launches = 0;
+  // options of the forward being launched: GEMM pipeline wait limit (0 =
+  // default) and the test stall of the gate/up GEMM
+  uint64_t fwd_wait_ns = 0;
+  bool fwd_stall = false;
   std::string last_error;
   // per-phase profiling
   std::vector<cudaEvent_t> prof_events;

@@ -15,6 +15,10 @@
 // bitmaps, status word); the partial logits are fully overwritten. Two calls
 // whose work overlaps on the GPU (different streams without ordering, or
 // several host threads) race on the array and must not be issued.
+// The top-k kernel's status word (set for NaN keys, which then get the
+// smallest untaken expert ids) lives in the array too and is not read back:
+// this call returns without waiting for the GPU, so it reports host-side
+// argument errors only.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -72,6 +76,10 @@ extern "C" moe_status_t moe_router_topk_noalloc(const void* x, int64_t T,
   if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(router_weight)) & 15)
     return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
+  // the partial logits alone take 4 * T * E bytes: larger T cannot fit, and
+  // rejecting it here keeps the size arithmetic below far from overflow
+  if (T > static_cast<int64_t>(kScratchBytes / (4 * static_cast<size_t>(n_routed_experts))))
+    return MOE_ERR_INVALID_ARG;
 
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;

@@ -14,8 +14,9 @@
 //   which keeps the result deterministic.
 // Kernel 2 (router_topk_kernel): one warp per token. Lane l holds experts
 //   l, l+32, ...; it adds the partials, takes the sigmoid, forms the key
-//   score + bias, and the warp extracts the k largest keys (ties to the lower
-//   expert index) by k rounds of a shuffle arg-max. The weights use the
+//   score + bias, applies the group filter when n_group > 1 (below), and the
+//   warp extracts the k largest keys (ties to the lower expert index) by k
+//   rounds of a shuffle arg-max. The weights use the
 //   unbiased scores: w = score / sum(selected scores) * 2.827. It also counts
 //   tokens per expert and sets the token's bit in the expert's bitmap, which
 //   the dispatch uses to place each (token, slot) pair.
@@ -130,12 +131,71 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const __nv_bfloat16*
 
 constexpr int kPerLane = kMaxExperts / 32;
 
+// Group-limited routing (n_group > 1; "Kimi K2 Base" raw config fields
+// n_group / topk_group, both 1 for K2, whose config post, §2.4, explains what
+// grouping is for). The experts form n_group contiguous groups of E / n_group;
+// a group scores the fp32 sum of its two largest keys (its one key for groups
+// of one); the topk_group best groups are kept, ties to the lower group; the
+// other groups' keys become -inf so that the top-k below never picks them.
+// One warp: the keys go through this warp's shared-memory row, lane g < n_group
+// scans group g, and the groups are picked by topk_group shuffle arg-max rounds.
+__device__ __forceinline__ void group_filter(float (&key)[kMaxExperts / 32], int E, int n_group,
+                                             int topk_group, float* __restrict__ row,
+                                             int lane) {
+  const unsigned full = 0xffffffffu;
+#pragma unroll
+  for (int i = 0; i < kMaxExperts / 32; ++i)
+    if (lane + 32 * i < E) row[lane + 32 * i] = key[i];
+  __syncwarp();
+  const int gs = E / n_group;
+  float gscore = -INFINITY;
+  if (lane < n_group) {
+    float b1 = -INFINITY, b2 = -INFINITY;  // the two largest keys of group `lane`
+    for (int j = 0; j < gs; ++j) {
+      const float v = row[lane * gs + j];
+      if (v > b1) {
+        b2 = b1;
+        b1 = v;
+      } else if (v > b2) {
+        b2 = v;
+      }
+    }
+    gscore = gs >= 2 ? b1 + b2 : b1;
+  }
+  uint32_t kept = 0;  // bit g: group g kept
+  for (int r = 0; r < topk_group; ++r) {
+    float bv = (lane < n_group && !((kept >> lane) & 1u)) ? gscore : -INFINITY;
+    int bi = (lane < n_group && !((kept >> lane) & 1u)) ? lane : 0x7fffffff;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(full, bv, off);
+      const int oi = __shfl_xor_sync(full, bi, off);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if (bi >= n_group) {  // NaN or -inf scores only: the lowest group not yet kept
+      bi = 0;
+      while (bi < n_group && ((kept >> bi) & 1u)) ++bi;
+    }
+    kept |= 1u << bi;
+  }
+#pragma unroll
+  for (int i = 0; i < kMaxExperts / 32; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E && !((kept >> (e / gs)) & 1u)) key[i] = -INFINITY;
+  }
+  __syncwarp();
+}
+
 __global__ void __launch_bounds__(256) router_topk_kernel(
     const float* __restrict__ part, int splits, const float* __restrict__ bias, int T, int E,
     int k, float scale, int norm, const int32_t* __restrict__ forced, int32_t* __restrict__ ids,
     float* __restrict__ wts, int32_t* __restrict__ counts, uint32_t* __restrict__ bitmap,
     int W, uint32_t* __restrict__ status, int32_t* __restrict__ ids_out,
-    float* __restrict__ wts_out, float* __restrict__ logits_out) {
+    float* __restrict__ wts_out, float* __restrict__ logits_out, int n_group, int topk_group) {
+  __shared__ float group_rows[256 / 32][kMaxExperts];  // one key row per warp (group filter)
   const int lane = threadIdx.x & 31;
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= T) return;
@@ -203,6 +263,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     }
   }
   if (!use_forced) {
+    if (n_group > 1) group_filter(key, E, n_group, topk_group, group_rows[threadIdx.x >> 5], lane);
     uint32_t taken = 0;  // bit i: expert lane + 32 i already chosen
     for (int j = 0; j < k; ++j) {
       float bk = -INFINITY;
@@ -333,7 +394,7 @@ cudaError_t launch_router_topk(moe_handle* h, int T, int splits, const int32_t* 
   router_topk_kernel<<<blocks, 256, 0, s>>>(
       h->ws.logits_part, splits, h->w.bias, T, dm.E, dm.k, h->cfg.routed_scaling_factor,
       h->cfg.norm_topk_prob, forced, h->ws.ids, h->ws.wts, h->ws.counts, h->ws.bitmap, W,
-      h->ws.status, ids_out, wts_out, logits_out);
+      h->ws.status, ids_out, wts_out, logits_out, h->cfg.n_group, h->cfg.topk_group);
   h->launches++;
   return cudaGetLastError();
 }
@@ -355,7 +416,7 @@ cudaError_t launch_router_raw(const void* x, const float* router_weight, const f
   const int blocks = (T * 32 + 255) / 256;
   router_topk_kernel<<<blocks, 256, 0, s>>>(part, splits, bias, T, E, k, scale, norm, nullptr, ids,
                                             wts, counts, bitmap, W, status, nullptr, nullptr,
-                                            nullptr);
+                                            nullptr, 1, 1);
   return cudaGetLastError();
 }
 

@@ -61,9 +61,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete. Returns false when
-// the wait ran out of time or *abort (if given) became non-zero.
+// the wait ran out of time (limit_ns) or *abort (if given) became non-zero.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile uint32_t* abort) {
+                                          volatile uint32_t* abort,
+                                          uint64_t limit_ns = kTimeoutNs) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait(addr, parity)) return true;
   const uint64_t t0 = globaltimer();
@@ -71,7 +72,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
     if (mbar_try_wait(addr, parity)) return true;
     if ((i & 31u) == 0) {
       if (abort != nullptr && *abort) return false;
-      if (globaltimer() - t0 > kTimeoutNs) return false;
+      if (globaltimer() - t0 > limit_ns) return false;
     }
   }
 }
@@ -213,7 +214,8 @@ __device__ __forceinline__ void st_shared_remote_u32(void* p, uint32_t cta, uint
 // mbar_wait with cluster-scope acquire: for phases completed by arrivals from
 // the other CTA of the pair that publish data in shared memory.
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
-                                                  volatile uint32_t* abort) {
+                                                  volatile uint32_t* abort,
+                                                  uint64_t limit_ns = kTimeoutNs) {
   const uint32_t addr = smem_u32(bar);
   const uint64_t t0 = globaltimer();
   for (uint32_t i = 0;; ++i) {
@@ -228,7 +230,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
     if (ok) return true;
     if ((i & 31u) == 31u) {
       if (abort != nullptr && *abort) return false;
-      if (globaltimer() - t0 > kTimeoutNs) return false;
+      if (globaltimer() - t0 > limit_ns) return false;
     }
   }
 }

@@ -50,8 +50,10 @@ def test_config_defaults_are_k2(smoe):
 
 
 @pytest.mark.parametrize("field,value,expect", [
-    ("n_group", 8, "MOE_ERR_UNSUPPORTED"),
-    ("topk_group", 4, "MOE_ERR_UNSUPPORTED"),
+    ("n_group", 64, "MOE_ERR_UNSUPPORTED"),       # more groups than warp lanes
+    ("n_group", 5, "MOE_ERR_INVALID_ARG"),        # 384 experts do not split into 5 groups
+    ("n_group", 0, "MOE_ERR_INVALID_ARG"),
+    ("topk_group", 4, "MOE_ERR_INVALID_ARG"),     # more kept groups than groups (n_group 1)
     ("hidden_size", 7000, "MOE_ERR_UNSUPPORTED"),
     ("moe_intermediate_size", 100, "MOE_ERR_UNSUPPORTED"),
     ("n_routed_experts", 1024, "MOE_ERR_UNSUPPORTED"),
@@ -71,6 +73,19 @@ def test_create_rejects_bad_configs_before_touching_a_device(smoe, field, value,
     with pytest.raises(smoe.MoeError) as ei:
         smoe.moe_create(c, 0)
     assert ei.value.status == getattr(smoe, expect)
+
+
+def test_group_limited_configs_are_checked_before_touching_a_device(smoe):
+    """n_group > 1: the kept groups must hold at least k experts (here 48
+    groups of 8 with one kept cannot supply 9 experts)."""
+    c = smoe.moe_config_init_k2(n_group=48, topk_group=1, num_experts_per_tok=9)
+    with pytest.raises(smoe.MoeError) as ei:
+        smoe.moe_create(c, 0)
+    assert ei.value.status == smoe.MOE_ERR_UNSUPPORTED  # n_group > 32 comes first
+    c = smoe.moe_config_init_k2(n_group=32, topk_group=1, num_experts_per_tok=13)
+    with pytest.raises(smoe.MoeError) as ei:
+        smoe.moe_create(c, 0)
+    assert ei.value.status == smoe.MOE_ERR_INVALID_ARG  # 1 group of 12 < 13 experts
 
 
 @pytest.mark.parametrize("E,k,ns,expect", [

@@ -23,7 +23,7 @@ int main(void) {
   if (moe_config_init_k2(&c) != MOE_OK) return 1;
   if (c.hidden_size != 7168 || c.n_routed_experts != 384 || c.num_experts_per_tok != 8) return 2;
   if (moe_config_init_k2(NULL) != MOE_ERR_INVALID_ARG) return 3;
-  c.n_group = 8; /* rejected before any device call */
+  c.n_group = 64; /* rejected before any device call */
   moe_handle_t* h = NULL;
   if (moe_create(&c, 0, &h) != MOE_ERR_UNSUPPORTED || h != NULL) return 4;
   if (strcmp(moe_status_string(MOE_OK), "ok") != 0) return 5;
@@ -32,7 +32,8 @@ int main(void) {
          offsetof(moe_config_t, routed_scaling_factor), offsetof(moe_config_t, weight_block_size),
          offsetof(moe_config_t, max_tokens));
   printf("weights %zu %zu\n", sizeof(moe_weights_t), offsetof(moe_weights_t, shared_down_scale));
-  printf("opts %zu %zu\n", sizeof(moe_forward_opts_t), offsetof(moe_forward_opts_t, flags));
+  printf("opts %zu %zu %zu %zu\n", sizeof(moe_forward_opts_t), offsetof(moe_forward_opts_t, flags),
+         offsetof(moe_forward_opts_t, pair_rows_out), offsetof(moe_forward_opts_t, wait_limit_ns));
   return 0;
 }
 """
@@ -64,4 +65,5 @@ def test_header_is_c99_and_layouts_match_the_binding(smoe, tmp_path):
     assert got["config"] == [ctypes.sizeof(C), C.routed_scaling_factor.offset,
                              C.weight_block_size.offset, C.max_tokens.offset]
     assert got["weights"] == [ctypes.sizeof(W), W.shared_down_scale.offset]
-    assert got["opts"] == [ctypes.sizeof(O), O.flags.offset]
+    assert got["opts"] == [ctypes.sizeof(O), O.flags.offset, O.pair_rows_out.offset,
+                           O.wait_limit_ns.offset]
