@@ -83,7 +83,9 @@ def test_dense_workload_and_its_counts():
     T = 64
     a = bench.algorithmic(s, T, "bf16", np.zeros((T, 0), np.int64))
     assert a["U"] == 0
-    assert a["gemm_gate_up"][0] == 2 * 18432 * 7168 * 2 + T * 9 * (7168 + 2048) * 2
+    # gate/up: the weights once, x once per token (not per gathered row), h
+    # once per row
+    assert a["gemm_gate_up"][0] == 2 * 18432 * 7168 * 2 + T * 7168 * 2 + T * 9 * 2048 * 2
     assert a["gemm_gate_up"][1] == 2 * T * 2 * 18432 * 7168
     assert a["gemm_down"][1] == 2 * T * 18432 * 7168
     # down: the weights once, h rows in, BF16 per-row outputs out
