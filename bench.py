@@ -8,7 +8,9 @@ batch of T synthetic tokens with weights resident in HBM. Prints one JSON
 line (rank 0).
 
 Workloads (--config):
-  decode      K2 layer, T = 64 tokens, BF16 experts (default)
+  decode      K2 layer, T = 64 tokens, BF16 experts (default); the line also
+              carries a "prefill" key: the same measurement at T = 8192 on
+              the same weights and handle (--no-prefill leaves it out)
   prefill     K2 layer, T = 8192 tokens, BF16 experts
   fp8-T<n>    K2 layer, T = n tokens, FP8 e4m3 experts with 128x128 scales
   dense-T<n>  K2's dense FFN layer (its first layer: one SwiGLU MLP of
@@ -49,6 +51,7 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "K2 MoE layer tokens/s; % of HBM (decode) / tensor-peak (prefill) roofline"
+PREFILL_T = 8192
 UNIT = "tokens/s"
 PHASES = ("router_logits", "router_topk", "route_scan", "dispatch", "gemm_gate_up",
           "gemm_down", "combine")
@@ -60,7 +63,8 @@ KERNEL_SOURCES = {"gemm_gate_up": _GEMM_SOURCES, "gemm_down": _GEMM_SOURCES}
 # ----------------------------------------------------------------- workloads
 def workload(name: str):
     if name == "decode":
-        return dict(T=64, fmt="bf16", desc="K2 MoE layer decode step, T=64 tokens, BF16 experts")
+        return dict(T=64, fmt="bf16", with_prefill=True,
+                    desc="K2 MoE layer decode step, T=64 tokens, BF16 experts")
     if name == "prefill":
         return dict(T=8192, fmt="bf16", desc="K2 MoE layer prefill, T=8192 tokens, BF16 experts")
     if name.startswith("dense-"):
@@ -236,25 +240,33 @@ def np_expert(mats: dict) -> dict:
 
 # -------------------------------------------------------------------- arms
 def algorithmic(shape, T, fmt, ids: np.ndarray):
-    """Algorithmic bytes and flops of each GEMM launch for the actual routing."""
+    """Algorithmic bytes and flops of each GEMM launch, and of the layer, for
+    the actual routing. x counts once per token (T rows, the method's input;
+    the gathered copy per (token, slot) is this library's intermediate), h
+    once per routed row (written by gate/up, read by down), the per-row
+    outputs once per routed row (BF16, read by the combine)."""
     d, f, E, k, ns = (shape.hidden_size, shape.moe_intermediate_size, shape.n_routed_experts,
                       shape.num_experts_per_tok, shape.n_shared_experts)
     wb = 1 if fmt == "fp8" else 2
-    U = len(np.unique(ids))
+    U = len(np.unique(ids)) if E > 0 else 0
     G_used = U + ns
     R = T * (k + ns)
     sb = lambda r, c: (r // 128) * (c // 128) * 4 if fmt == "fp8" else 0
-    gate_up_bytes = G_used * 2 * (f * d * wb + sb(f, d)) + R * d * wb + R * f * wb
+    gate_up_bytes = G_used * 2 * (f * d * wb + sb(f, d)) + T * d * wb + R * f * wb
     down_bytes = G_used * (d * f * wb + sb(d, f)) + R * f * wb + R * d * 2  # BF16 row outputs
     if fmt == "fp8":
-        gate_up_bytes += R * (d // 128) * 4 + R * (f // 128) * 4
+        gate_up_bytes += T * (d // 128) * 4 + R * (f // 128) * 4
         down_bytes += R * (f // 128) * 4
     gate_up_flops = 2 * R * 2 * f * d
     down_flops = 2 * R * d * f
-    layer_bytes = G_used * 3 * (d * f * wb) + E * d * 4 + E * 4 + T * d * 2 * 2
+    layer_bytes = G_used * 3 * (d * f * wb + sb(d, f)) + E * d * 4 + E * 4 + T * d * 2 * 2
     layer_flops = 2 * R * 3 * d * f + 2 * T * E * d
     return dict(U=U, gemm_gate_up=(gate_up_bytes, gate_up_flops),
                 gemm_down=(down_bytes, down_flops), layer=(layer_bytes, layer_flops))
+
+
+# datasheet figures (dense, HGX B200) beside the measured ones
+DATASHEET = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
 
 def kernel_src_hash(kernel: str) -> str:
@@ -276,54 +288,19 @@ def traffic_for(kernel: str, config: str):
     return j.get("bytes_per_launch")
 
 
-def run_native(args, wl):
-    import sparse_moe_sigmoid_b200 as smoe
+def measure(smoe, h, x, y, T, fmt, shape, args, dev, config_name):
+    """Time K plain forwards of T tokens (after W warm-ups), then the same
+    forwards with the library's phase events, then end to end from pinned
+    host memory. Returns the measurement as a dict (max over ranks)."""
     ws, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if ws > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-    shape, T, fmt = wl.get("shape", synth.K2), wl["T"], wl["fmt"]
-    x = synth.make_tokens(shape, T, device=dev)
-    Wg, b = synth.make_router(shape, device=dev)
-    ew = synth.make_experts(shape, device=dev, fmt=fmt)
-    cfg = smoe.moe_config_init_k2(
-        max_tokens=T, n_routed_experts=shape.n_routed_experts,
-        num_experts_per_tok=shape.num_experts_per_tok, n_shared_experts=shape.n_shared_experts,
-        weight_format=smoe.MOE_WEIGHT_BF16 if fmt == "bf16" else smoe.MOE_WEIGHT_FP8_E4M3_BLOCK)
-    h = smoe.moe_create(cfg, local)
-    smoe.moe_load_weights(h, Wg, b, ew.gate, ew.up, ew.down, ew.shared_gate, ew.shared_up,
-                          ew.shared_down, ew.gate_scale, ew.up_scale, ew.down_scale,
-                          ew.shared_gate_scale, ew.shared_up_scale, ew.shared_down_scale)
-    y = torch.empty_like(x)
-    ids = torch.empty((T, shape.num_experts_per_tok), dtype=torch.int32, device=dev)
-    smoe.moe_forward(h, x, y, topk_ids_out=ids, flags=smoe.MOE_FLAG_SYNC_CHECK)
-    ids_np = ids.cpu().numpy()
-
-    # CPU oracle baseline (rank 0, one GPU only), before the caller copies go
-    cpu = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        n_tok = 4 if T <= 64 else 3
-        ors = OracleSample(shape, T, fmt, n_tok, x.cpu(), Wg.cpu(), b.cpu(),
-                           lambda e: np_expert(synth.expert_slice(ew, e) if e >= 0
-                                               else synth.shared_slice(ew)))
-        t0 = time.perf_counter()
-        n, reps = 0, 0
-        while True:
-            n += ors.run_once()
-            reps += 1
-            if time.perf_counter() - t0 > 10.0 or reps >= 20:
-                break
-        el = time.perf_counter() - t0
-        cpu = {"value": n / el, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{ors.describe()}; {reps} repetitions in {el:.1f} s"}
-    del ew
-    torch.cuda.empty_cache()
-
     stream = torch.cuda.current_stream()
+    ids = torch.empty((T, max(shape.num_experts_per_tok, 1)), dtype=torch.int32, device=dev)
+    if shape.n_routed_experts > 0:
+        smoe.moe_forward(h, x, y, topk_ids_out=ids, flags=smoe.MOE_FLAG_SYNC_CHECK)
+        ids_np = ids.cpu().numpy()
+    else:
+        smoe.moe_forward(h, x, y, flags=smoe.MOE_FLAG_SYNC_CHECK)
+        ids_np = np.zeros((T, 0), np.int64)
     for _ in range(args.warmup):
         smoe.moe_forward(h, x, y)
     torch.cuda.synchronize()
@@ -391,50 +368,136 @@ def run_native(args, wl):
     dom_name = PHASES[dom]
     alg = algorithmic(shape, T, fmt, ids_np)
     peaks = load_peaks()
+    ten_peak = peaks["bf16_sus"] * (2.0 if fmt == "fp8" else 1.0)
+    ten_sheet = DATASHEET["bf16_tflops"] * (2.0 if fmt == "fp8" else 1.0)
     byts, flops = alg.get(dom_name, alg["layer"])
     dur = mean_ph[dom] / 1e3
     hbm_t = byts / (peaks["hbm"] * 1e9)
-    ten_t = flops / (peaks["bf16_sus"] * 1e12 * (2.0 if fmt == "fp8" else 1.0))
+    ten_t = flops / (ten_peak * 1e12)
     if hbm_t >= ten_t:
         roof = {"bound": "hbm", "achieved": byts / dur / 1e9, "peak": peaks["hbm"],
                 "unit": "GB/s"}
     else:
-        roof = {"bound": "tensor", "achieved": flops / dur / 1e12,
-                "peak": peaks["bf16_sus"] * (2.0 if fmt == "fp8" else 1.0), "unit": "TFLOP/s"}
+        roof = {"bound": "tensor", "achieved": flops / dur / 1e12, "peak": ten_peak,
+                "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = traffic_for(dom_name, args.config)
+    roof["traffic"] = traffic_for(dom_name, config_name)
     roof.update({
         "kernel": dom_name, "launch_ms": round(mean_ph[dom], 4),
         "algorithmic_bytes": int(byts), "algorithmic_flops": int(flops),
         "hbm_frac": (byts / dur / 1e9) / peaks["hbm"],
-        "tensor_frac": (flops / dur / 1e12) / (peaks["bf16_sus"] * (2.0 if fmt == "fp8" else 1.0)),
+        "tensor_frac": (flops / dur / 1e12) / ten_peak,
+        "hbm_frac_datasheet": (byts / dur / 1e9) / DATASHEET["hbm_gbs"],
+        "tensor_frac_datasheet": (flops / dur / 1e12) / ten_sheet,
         "peak_source": f"{peaks['src']} (HBM copy GB/s; sustained cuBLAS bf16 TF/s"
-                       f"{', x2 nominal fp8 ratio' if fmt == 'fp8' else ''})"})
+                       f"{', x2 nominal fp8 ratio' if fmt == 'fp8' else ''}); the *_datasheet "
+                       f"fractions use 8 TB/s and {ten_sheet:.0f} TF/s dense"})
     layer_bytes, layer_flops = alg["layer"]
+    sec = ms_max / 1e3
+    return {
+        "T": T, "value": value, "ms_per_step": ms_max, "U": alg["U"],
+        "roofline": roof,
+        "layer_roofline": {
+            "bytes": int(layer_bytes), "flops": int(layer_flops),
+            "hbm_frac": (layer_bytes / sec / 1e9) / peaks["hbm"],
+            "tensor_frac": (layer_flops / sec / 1e12) / ten_peak,
+            "hbm_frac_datasheet": (layer_bytes / sec / 1e9) / DATASHEET["hbm_gbs"],
+            "tensor_frac_datasheet": (layer_flops / sec / 1e12) / ten_sheet},
+        "phases_ms": {p: round(float(v), 4) for p, v in zip(PHASES, mean_ph)},
+        "e2e": {"value": tokens_all / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": int(xh.numel() * 2),
+                "d2h_bytes_per_step": int(yh.numel() * 2), "ms_per_step": e2e_ms,
+                "api": "moe_forward_host_async + moe_host_wait (pinned host x and y; uploads "
+                       "and downloads overlap neighbouring forwards)"},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+
+
+def run_native(args, wl):
+    import sparse_moe_sigmoid_b200 as smoe
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    shape, T, fmt = wl.get("shape", synth.K2), wl["T"], wl["fmt"]
+    # the default (decode) line also measures prefill on the same weights
+    T_pre = PREFILL_T if (wl.get("with_prefill") and not args.no_prefill) else 0
+    T_max = max(T, T_pre)
+    x_all = synth.make_tokens(shape, T_max, device=dev)
+    x = x_all[:T].contiguous()
+    Wg, b = synth.make_router(shape, device=dev)
+    ew = synth.make_experts(shape, device=dev, fmt=fmt)
+    cfg = smoe.moe_config_init_k2(
+        max_tokens=T_max, n_routed_experts=shape.n_routed_experts,
+        num_experts_per_tok=shape.num_experts_per_tok, n_shared_experts=shape.n_shared_experts,
+        weight_format=smoe.MOE_WEIGHT_BF16 if fmt == "bf16" else smoe.MOE_WEIGHT_FP8_E4M3_BLOCK)
+    h = smoe.moe_create(cfg, local)
+    smoe.moe_load_weights(h, Wg, b, ew.gate, ew.up, ew.down, ew.shared_gate, ew.shared_up,
+                          ew.shared_down, ew.gate_scale, ew.up_scale, ew.down_scale,
+                          ew.shared_gate_scale, ew.shared_up_scale, ew.shared_down_scale)
+    torch.cuda.synchronize()
+
+    # CPU oracle baseline (rank 0, one GPU only), before the caller copies go
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        n_tok = 4 if T <= 64 else 3
+        ors = OracleSample(shape, T, fmt, n_tok, x.cpu(), Wg.cpu(), b.cpu(),
+                           lambda e: np_expert(synth.expert_slice(ew, e) if e >= 0
+                                               else synth.shared_slice(ew)))
+        t0 = time.perf_counter()
+        n, reps = 0, 0
+        while True:
+            n += ors.run_once()
+            reps += 1
+            if time.perf_counter() - t0 > 10.0 or reps >= 20:
+                break
+        el = time.perf_counter() - t0
+        cpu = {"value": n / el, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{ors.describe()}; {reps} repetitions in {el:.1f} s"}
+    del ew
+    torch.cuda.empty_cache()
+
+    y = torch.empty_like(x)
+    m = measure(smoe, h, x, y, T, fmt, shape, args, dev, args.config)
+    pre = None
+    if T_pre:
+        xp = x_all[:T_pre].contiguous()
+        pre = measure(smoe, h, xp, torch.empty_like(xp), T_pre, fmt, shape, args, dev, "prefill")
+        pre = {"workload": f"K2 MoE layer prefill, T={T_pre} tokens, {fmt.upper()} experts "
+                           "(same weights and handle)",
+               "ms_per_step": pre["ms_per_step"], "value": pre["value"], "unit": UNIT,
+               "roofline": pre["roofline"], "layer_roofline": pre["layer_roofline"],
+               "phases_ms": pre["phases_ms"], "e2e": pre["e2e"],
+               "gpu_launches": pre["gpu_launches"], "clocks": pre["clocks"],
+               "distinct_experts_hit": pre["U"]}
     out = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+        "metric": METRIC, "value": m["value"], "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if fmt == "bf16" else "e4m3",
         "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) weights, random init)",
         "config": {"workload": wl["desc"], "tokens": T, "global_batch": T * ws,
                    "hidden_size": shape.hidden_size, "n_routed_experts": shape.n_routed_experts,
-                   "top_k": shape.num_experts_per_tok, "n_shared_experts": shape.n_shared_experts, "moe_intermediate_size":
-                       shape.moe_intermediate_size, "parallelism": f"replicas x{ws}",
-                   "distinct_experts_hit": alg["U"],
+                   "top_k": shape.num_experts_per_tok, "n_shared_experts": shape.n_shared_experts,
+                   "moe_intermediate_size": shape.moe_intermediate_size,
+                   "parallelism": f"replicas x{ws}", "distinct_experts_hit": m["U"],
                    "l2": "no flush: the expert weights streamed each step exceed the 126 MB L2"},
-        "roofline": roof,
-        "layer_roofline": {"bytes": int(layer_bytes), "flops": int(layer_flops),
-                           "hbm_frac": (layer_bytes / (ms_max / 1e3) / 1e9) / peaks["hbm"]},
-        "phases_ms": {p: round(float(v), 4) for p, v in zip(PHASES, mean_ph)},
+        "roofline": m["roofline"],
+        "layer_roofline": m["layer_roofline"],
+        "phases_ms": m["phases_ms"],
         "cpu_baseline": cpu,
-        "e2e": {"value": tokens_all / (e2e_ms / 1e3), "unit": UNIT,
-                "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 2),
-                "ms_per_step": e2e_ms,
-                "api": "moe_forward_host_async + moe_host_wait (pinned host x and y; uploads and "
-                       "downloads overlap neighbouring forwards)"},
-        "gpu_launches": int(launches),
-        "clocks": clk,
+        "e2e": m["e2e"],
+        "gpu_launches": m["gpu_launches"] + (pre["gpu_launches"] if pre else 0),
+        "clocks": m["clocks"],
     }
+    if pre:
+        out["prefill"] = pre
+        out["gpu_launches_note"] = ("kernels launched in the timed regions of the decode line "
+                                    "and of the prefill key together")
     smoe.moe_destroy(h)
     if ws > 1:
         import torch.distributed as dist
@@ -486,6 +549,8 @@ def main(argv=None):
     ap.add_argument("--config", default="decode")
     ap.add_argument("--impl", default="native", choices=("native", "reference"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="decode line only (no prefill key)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (small profiling cases)")
     ap.add_argument("--experts", type=int, default=None,
