@@ -362,13 +362,19 @@ moe_status_t moe_create(const moe_config_t* cfg, int device, moe_handle_t** out)
   }
   for (int i = 0; i < 16 && ok; ++i) {
     const uint32_t bn = 16u * (i + 1);
+    uint32_t box[2] = {kbox, bn};
     uint64_t dx[2] = {d, Rm};
     uint64_t sx[1] = {d * wb};
-    uint32_t box[2] = {kbox, bn};
     ok = ok && smoe::make_tmap(&h->tm_xp[i], dt, 2, h->ws.xp, dx, sx, box, &why);
     uint64_t dh[2] = {f, Rm};
     uint64_t sh[1] = {f * wb};
     ok = ok && smoe::make_tmap(&h->tm_h[i], dt, 2, h->ws.hbuf, dh, sh, box, &why);
+  }
+  if (dm.fp8 && ok) {  // gathers of quantised token rows, rows [0, T) of xp (one-row box)
+    uint64_t dx[2] = {d, Rm};
+    uint64_t sx[1] = {d};
+    uint32_t box[2] = {kbox, 1};
+    ok = smoe::make_tmap(&h->tm_xg, dt, 2, h->ws.xp, dx, sx, box, &why);
   }
   if (!ok) {
     free_all(h);
@@ -519,6 +525,16 @@ moe_status_t launch_forward(moe_handle* h, const void* x, int64_t T, void* y,
     }
   } reset{h};
 
+  if (!dm.fp8 && p1.gather) {  // the gate/up GEMM gathers token rows straight from x
+    uint64_t dx[2] = {static_cast<uint64_t>(dm.d), static_cast<uint64_t>(T)};
+    uint64_t sx[1] = {static_cast<uint64_t>(dm.d) * 2};
+    uint32_t box[2] = {64, 1};
+    std::string why;
+    if (!smoe::make_tmap(&h->tm_xg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dx,
+                         sx, box, &why))
+      return fail(h, MOE_ERR_CUDA, why);
+  }
+
   mark(0);
   CUDA_TRY(h, cudaMemsetAsync(h->ws.sched, 0, h->ws.zero_bytes, s), "clear counts");
   // without routed experts (a dense FFN layer) there is nothing to route: the
@@ -543,7 +559,7 @@ moe_status_t launch_forward(moe_handle* h, const void* x, int64_t T, void* y,
   mark(2);
   CUDA_TRY(h, smoe::launch_route_scan(h, Ti, p1, p2, s), "route scan launch");
   mark(3);
-  CUDA_TRY(h, smoe::launch_dispatch(h, x, Ti, s), "dispatch launch");
+  CUDA_TRY(h, smoe::launch_dispatch(h, x, Ti, p1.gather, s), "dispatch launch");
   if (opts && opts->expert_offsets_out && dm.E > 0)
     CUDA_TRY(h, cudaMemcpyAsync(opts->expert_offsets_out, h->ws.offsets, (dm.E + 1) * 4,
                                 cudaMemcpyDeviceToDevice, s),

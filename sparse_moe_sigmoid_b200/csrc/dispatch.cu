@@ -14,9 +14,11 @@
 //   into offsets; the GEMM work-unit prefix for both grouped GEMMs; and for
 //   every expert the running popcount of its token bitmap words, so a pair's
 //   rank inside its expert is one popcount away.
-// dispatch_kernel: one warp per row. It places the pair (pair_row,
-//   row_token) and copies the token's x row into the gathered matrix with
-//   16-byte loads and stores. In the FP8 format it quantises on the way:
+// dispatch: places every (token, slot) pair (pair_row, row_token). For row
+//   tiles up to kGatherMaxBn rows the gate/up GEMMs gather each tile's token
+//   rows straight from x with TMA (tile::gather4), so nothing is copied
+//   (FP8: each token's x row is quantised once); taller tiles read the rows
+//   copied here into expert order (FP8: quantised per row). Quantisation:
 //   per 128 columns s = amax/448 and q = e4m3(x/s), both divisions
 //   correctly rounded, conversion nearest-even and saturating.
 // combine_kernel: y[t] = sum_j w[t,j] * out[row(t,j)] + sum_s out[shared
@@ -59,6 +61,7 @@ GemmPlan plan_gate_up(const Dims& dm, int64_t T) {
   p.bn = dm.fp8 ? pick_bn(want, fp8_bn, 4) : pick_bn(want, bf16_bn, 9);
   p.na = 2;
   p.pair = !dm.fp8 && pair_bn_supported(p.bn) && dm.f % 256 == 0;
+  p.gather = !p.pair && p.bn <= kGatherMaxBn;
   p.m_tiles = dm.f / (p.pair ? 256 : kBlock);
   p.k_blocks = dm.fp8 ? dm.d / 128 : dm.d / 64;
   return p;
@@ -76,6 +79,7 @@ GemmPlan plan_down(const Dims& dm, int64_t T) {
   GemmPlan p;
   p.bn = dm.fp8 ? pick_bn(want, fp8_bn, 5) : pick_bn(want, bf16_bn, 9);
   p.pair = !dm.fp8 && pair_bn_supported(p.bn) && dm.d % 256 == 0 && dm.f % 128 == 0;
+  p.gather = false;  // h rows are written in expert order by gate/up
   // two weight tiles per unit: FP8 up to 64 rows (measured: T=128 down GEMM
   // 1.05 -> 0.80 ms); BF16 from 64 rows (at 16 rows it changed nothing)
   p.na = (!p.pair && dm.d % 256 == 0 && (dm.fp8 ? p.bn <= 64 : p.bn >= 64)) ? 2 : 1;
@@ -173,27 +177,6 @@ __device__ __forceinline__ int place_row(int i, int T, int k, int E, const int32
   return offsets[E + s] + t;
 }
 
-__global__ void __launch_bounds__(256) dispatch_bf16_kernel(
-    const __nv_bfloat16* __restrict__ x, int T, int d, int k, int E, int items,
-    const int32_t* __restrict__ ids, const uint32_t* __restrict__ bitmap,
-    const int32_t* __restrict__ word_prefix, const int32_t* __restrict__ offsets, int W,
-    int32_t* __restrict__ pair_row, int32_t* __restrict__ row_token,
-    __nv_bfloat16* __restrict__ xp) {
-  const int lane = threadIdx.x & 31;
-  const int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (i >= items) return;
-  int t;
-  const int row = place_row(i, T, k, E, ids, bitmap, word_prefix, offsets, W, &t);
-  if (lane == 0) {
-    if (i < T * k) pair_row[i] = row;
-    row_token[row] = t;
-  }
-  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
-  uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)row * d);
-  const int n16 = d / 8;
-  for (int c = lane; c < n16; c += 32) dst[c] = __ldg(src + c);
-}
-
 // One row of d BF16 values -> d e4m3 codes + d/128 fp32 scales, by one warp:
 // each half-warp takes one 128-column group (16 lanes x 8 values).
 __device__ __forceinline__ void quant_row_e4m3(const __nv_bfloat16* __restrict__ src, int d,
@@ -239,6 +222,30 @@ __device__ __forceinline__ void quant_row_e4m3(const __nv_bfloat16* __restrict__
   }
 }
 
+// Tall row tiles: one warp per row places the pair (pair_row, row_token)
+// and copies the token's x row into the gathered matrix in row order with
+// 16-byte loads and stores (FP8: quantises it on the way, as below).
+__global__ void __launch_bounds__(256) dispatch_bf16_kernel(
+    const __nv_bfloat16* __restrict__ x, int T, int d, int k, int E, int items,
+    const int32_t* __restrict__ ids, const uint32_t* __restrict__ bitmap,
+    const int32_t* __restrict__ word_prefix, const int32_t* __restrict__ offsets, int W,
+    int32_t* __restrict__ pair_row, int32_t* __restrict__ row_token,
+    __nv_bfloat16* __restrict__ xp) {
+  const int lane = threadIdx.x & 31;
+  const int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (i >= items) return;
+  int t;
+  const int row = place_row(i, T, k, E, ids, bitmap, word_prefix, offsets, W, &t);
+  if (lane == 0) {
+    if (i < T * k) pair_row[i] = row;
+    row_token[row] = t;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+  uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)row * d);
+  const int n16 = d / 8;
+  for (int c = lane; c < n16; c += 32) dst[c] = __ldg(src + c);
+}
+
 __global__ void __launch_bounds__(256) dispatch_fp8_kernel(
     const __nv_bfloat16* __restrict__ x, int T, int d, int k, int E, int items,
     const int32_t* __restrict__ ids, const uint32_t* __restrict__ bitmap,
@@ -255,6 +262,33 @@ __global__ void __launch_bounds__(256) dispatch_fp8_kernel(
     row_token[row] = t;
   }
   quant_row_e4m3(x + (size_t)t * d, d, xq + (size_t)row * d, xs + (size_t)row * (d / 128), lane);
+}
+
+// Short row tiles: one thread per (token, slot) pair and per shared-group
+// row (blocks [0, place_blocks)) writes the pair's row (pair_row) and the
+// row's token (row_token), which the gate/up GEMMs use to gather x rows; no
+// row is copied. FP8: the blocks after those quantise each token's x row
+// once (one warp per token) into rows [0, T) of xq / xs, which the GEMMs
+// gather from instead of x.
+__global__ void __launch_bounds__(256) dispatch_kernel(
+    const __nv_bfloat16* __restrict__ x, int T, int d, int k, int E, int items, int place_blocks,
+    const int32_t* __restrict__ ids, const uint32_t* __restrict__ bitmap,
+    const int32_t* __restrict__ word_prefix, const int32_t* __restrict__ offsets, int W,
+    int32_t* __restrict__ pair_row, int32_t* __restrict__ row_token, uint8_t* __restrict__ xq,
+    float* __restrict__ xs) {
+  if (static_cast<int>(blockIdx.x) < place_blocks) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= items) return;
+    int t;
+    const int row = place_row(i, T, k, E, ids, bitmap, word_prefix, offsets, W, &t);
+    if (i < T * k) pair_row[i] = row;
+    row_token[row] = t;
+    return;
+  }
+  const int lane = threadIdx.x & 31;
+  const int t = ((blockIdx.x - place_blocks) * blockDim.x + threadIdx.x) >> 5;
+  if (t >= T) return;
+  quant_row_e4m3(x + (size_t)t * d, d, xq + (size_t)t * d, xs + (size_t)t * (d / 128), lane);
 }
 
 // Dynamic activation quantisation of a dense [rows, d] BF16 matrix.
@@ -276,21 +310,31 @@ cudaError_t launch_act_quant(const void* x, int64_t rows, int d, uint8_t* q, flo
   return cudaGetLastError();
 }
 
-cudaError_t launch_dispatch(moe_handle* h, const void* x, int T, cudaStream_t s) {
+cudaError_t launch_dispatch(moe_handle* h, const void* x, int T, bool gather, cudaStream_t s) {
   const Dims& dm = h->dims;
   const int W = static_cast<int>((dm.Tmax + 31) / 32);
   const int items = T * (dm.k + dm.ns);
-  const int blocks = static_cast<int>(((int64_t)items * 32 + 255) / 256);
-  if (dm.fp8) {
-    dispatch_fp8_kernel<<<blocks, 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), T, dm.d, dm.k, dm.E, items, h->ws.ids,
-        h->ws.bitmap, h->ws.word_prefix, h->ws.offsets, W, h->ws.pair_row, h->ws.row_token,
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  if (gather) {
+    const int place_blocks = (items + 255) / 256;
+    const int quant_blocks = dm.fp8 ? (T * 32 + 255) / 256 : 0;
+    dispatch_kernel<<<place_blocks + quant_blocks, 256, 0, s>>>(
+        xb, T, dm.d, dm.k, dm.E, items, place_blocks, h->ws.ids, h->ws.bitmap,
+        h->ws.word_prefix, h->ws.offsets, W, h->ws.pair_row, h->ws.row_token,
         static_cast<uint8_t*>(h->ws.xp), h->ws.xs);
   } else {
-    dispatch_bf16_kernel<<<blocks, 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), T, dm.d, dm.k, dm.E, items, h->ws.ids,
-        h->ws.bitmap, h->ws.word_prefix, h->ws.offsets, W, h->ws.pair_row, h->ws.row_token,
-        static_cast<__nv_bfloat16*>(h->ws.xp));
+    const int blocks = static_cast<int>(((int64_t)items * 32 + 255) / 256);
+    if (dm.fp8) {
+      dispatch_fp8_kernel<<<blocks, 256, 0, s>>>(
+          xb, T, dm.d, dm.k, dm.E, items, h->ws.ids, h->ws.bitmap, h->ws.word_prefix,
+          h->ws.offsets, W, h->ws.pair_row, h->ws.row_token, static_cast<uint8_t*>(h->ws.xp),
+          h->ws.xs);
+    } else {
+      dispatch_bf16_kernel<<<blocks, 256, 0, s>>>(
+          xb, T, dm.d, dm.k, dm.E, items, h->ws.ids, h->ws.bitmap, h->ws.word_prefix,
+          h->ws.offsets, W, h->ws.pair_row, h->ws.row_token,
+          static_cast<__nv_bfloat16*>(h->ws.xp));
+    }
   }
   h->launches++;
   return cudaGetLastError();

@@ -59,6 +59,7 @@ struct Bf16Cfg {
   static_assert(kTmemCols <= 512, "TMEM holds 512 columns");
   static_assert(kStages >= 2, "need at least two stages");
   static_assert(!SWIGLU || NA == 2, "SwiGLU needs the gate and up tiles");
+  static_assert(BN <= 256, "a gathered tile takes at most two gather4 per lane");
 };
 
 template <int BN, int NA, bool SWIGLU>
@@ -122,7 +123,8 @@ __global__ void __launch_bounds__(192, 1)
   const int total_units = total_units_of(args, BN);
   const uint64_t lim = wait_limit(args);
 
-  if (warp == 0) {
+  if (warp == 0 && args.row_token == nullptr) {
+    // B rows in a box of the tile's own rows: lane 0 alone waits and loads
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
@@ -148,6 +150,49 @@ __global__ void __launch_bounds__(192, 1)
         *abort_flag = 1;
         atomicOr(args.status, MOE_DEVICE_WAIT_TIMEOUT);
       }
+    }
+  } else if (warp == 0) {
+    // gathered B rows: lane 0 waits for a free stage and loads the weight
+    // tiles, then the lanes load the tile's token rows, four per
+    // tile::gather4, lane l taking rows 4l.. and 4(l + 32)..
+    uint32_t it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+      const Unit un = decode_unit(u, args, BN);
+      const int n = ((un.nvalid + 15) / 16) * 16;  // rows the MMA reads
+      int tok[2][4] = {};
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+        if (4 * (lane + 32 * q) < n)
+          gather_rows(args, un.row0, un.row0 + 4 * (lane + 32 * q), un.row0 + un.nvalid, tok[q]);
+      const uint32_t tx = C::kA * C::kNumA + n * 128;
+      for (int kb = 0; kb < args.k_blocks; ++kb, ++it) {
+        const int s = it % C::kStages;
+        const uint32_t ph = (it / C::kStages) & 1u;
+        if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        uint8_t* st = smem + s * C::kStage;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[s], tx);
+          tma_load_3d(st, &tmA0, &full[s], kb * 64, un.mt * kRowStep, un.g);
+          if (NA == 2)
+            tma_load_3d(st + C::kA, &tmA1, &full[s], kb * 64, un.mt * kRowStep + kRow1, un.g);
+        }
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int r = 4 * (lane + 32 * q);
+          if (r < n)
+            tma_gather4(st + C::kA * C::kNumA + r * 128, &tmB, &full[s], kb * 64, tok[q][0],
+                        tok[q][1], tok[q][2], tok[q][3]);
+        }
+        __syncwarp();
+        if (lane == 0) *issued = it + 1;
+      }
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      atomicOr(args.status, MOE_DEVICE_WAIT_TIMEOUT);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -295,7 +340,10 @@ cudaError_t launch_gemm_bf16(moe_handle* h, bool gated, const GemmPlan& p, cudaS
   if (gated) {
     a.out = h->ws.hbuf;
     a.ld = dm.f;
-    const CUtensorMap& b = h->tm_xp[bi];
+    // short tiles gather their token rows from x; taller ones read the rows
+    // the dispatch copied into expert order
+    a.row_token = p.gather ? h->ws.row_token : nullptr;
+    const CUtensorMap& b = p.gather ? h->tm_xg : h->tm_xp[bi];
     const CUtensorMap &g = h->tm_gate, &u = h->tm_up;
     switch (p.bn) {
       case 16: return launch_one<16, 2, true>(h, g, u, b, a, s);

@@ -43,6 +43,7 @@ struct GemmArgs {
   int b_k;                   // K extent of B; the K index into B is (k mod b_k)
   int m_valid;               // only output features < m_valid are stored
   int kpp;                   // promoted BF16 GEMM: stages accumulated in TMEM per promotion
+  int kpp_rest;              // the same for K slices after the first (0: kpp)
   int stages;                // promoted GEMM: shared-memory ring depth
   int32_t* sched;            // pair GEMM: unit counter, zero at launch (dynamic units); null: static
   int ksplit;                // single-group mode: K slices per tile (0 or 1: none); slice s
@@ -52,7 +53,20 @@ struct GemmArgs {
   int out_bf16;               // promoted GEMM, plain mode: outputs stored BF16 (else fp32)
   uint64_t wait_ns;           // limit of each pipeline wait (the wind-down keeps the default)
   int stall;                  // test hook: the MMA issuer waits on a barrier nothing signals
+  // gathered B (gate/up): row i of a tile is row row_token[row0 + i] of the B
+  // tensor (the token's x row), loaded four rows per tile::gather4; null: the
+  // B rows are the tile's own rows [row0, row0 + BN) of B (down, router)
+  const int32_t* row_token;
 };
+
+// Token rows of B for rows [r, r + 4) of a gathered tile whose valid rows end
+// at `end` (rows past it repeat the tile's first row: they are loaded so that
+// the MMA's N stays a multiple of 16, and their outputs are never stored).
+__device__ __forceinline__ void gather_rows(const GemmArgs& a, int row0, int r, int end,
+                                            int (&tok)[4]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) tok[j] = __ldg(a.row_token + (r + j < end ? r + j : row0));
+}
 
 // Limit of a pipeline wait: the caller's, or the default.
 __device__ __forceinline__ uint64_t wait_limit(const GemmArgs& a) {

@@ -87,6 +87,7 @@ struct PromCfg {
   static_assert(kTmemCols <= 512, "TMEM holds 512 columns");
   static_assert(kPBufs >= 2, "the promotion needs two partial buffers at least");
   static_assert(FP8 || !GATED, "the BF16 promoted GEMM is plain");
+  static_assert(!GATED || BN <= 128, "a gathered tile takes at most one gather4 per lane");
   // scale staging of FP8: activation scales [KB][BN] and weight scales [2][KB]
   static constexpr int scale_bytes(int kb) { return FP8 ? (kb * BN + 2 * kb) * 4 : 0; }
   static constexpr int stages(int kb) {
@@ -164,7 +165,11 @@ __global__ void __maxnreg__(prom_regs<NPG>())
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int KPP = FP8 ? 1 : args.kpp;  // stages accumulated per promotion
+  // stages accumulated in TMEM per promotion (FP8: every block, its scales
+  // differ); the router's K slices after the first use kpp_rest
+  auto kpp_of = [&](const Unit& un) {
+    return FP8 ? 1 : (un.split > 0 && args.kpp_rest > 0 ? args.kpp_rest : args.kpp);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -200,7 +205,8 @@ __global__ void __maxnreg__(prom_regs<NPG>())
   const int total_units = total_units_of(args, BN);
   const uint64_t lim = wait_limit(args);
 
-  if (warp == 0) {
+  if (warp == 0 && args.row_token == nullptr) {
+    // B rows in a box of the tile's own rows: lane 0 alone waits and loads
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
@@ -228,6 +234,44 @@ __global__ void __maxnreg__(prom_regs<NPG>())
         atomicOr(args.status, MOE_DEVICE_WAIT_TIMEOUT);
       }
     }
+  } else if (warp == 0) {
+    // gathered B rows (gate/up): lane 0 waits for a free stage and loads the
+    // weight tiles, then the lanes load the tile's token rows, four per
+    // tile::gather4 (at most 128 rows: one gather per lane)
+    uint32_t it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+      const Unit un = decode_unit(u, args, BN);
+      const int n = ((un.nvalid + 15) / 16) * 16;  // rows the MMA reads
+      int tok[4] = {};
+      if (4 * lane < n) gather_rows(args, un.row0, un.row0 + 4 * lane, un.row0 + un.nvalid, tok);
+      const uint32_t tx = C::kA * C::kNumA + n * 128;
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const int s = it % S;
+        const uint32_t ph = (it / S) & 1u;
+        if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        uint8_t* st = smem + s * C::kStage;
+        const int kc = (un.split * KB + kb) * C::kKPerStage;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[s], tx);
+          const int arow = DUAL ? un.mt * 256 : un.mt * 128;
+          tma_load_3d(st, &tmA0, &full[s], kc, arow, un.g);
+          if (C::kTwoA)
+            tma_load_3d(st + C::kA, &tmA1, &full[s], kc, arow + (DUAL ? 128 : 0), un.g);
+        }
+        if (4 * lane < n)
+          tma_gather4(st + C::kA * C::kNumA + 4 * lane * 128, &tmB, &full[s], kc % args.b_k,
+                      tok[0], tok[1], tok[2], tok[3]);
+        __syncwarp();
+        if (lane == 0) *issued = it + 1;
+      }
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      atomicOr(args.status, MOE_DEVICE_WAIT_TIMEOUT);
+    }
   } else if (warp == 1) {
     if (lane == 0) {
       uint32_t it = 0;   // stages consumed so far
@@ -238,6 +282,7 @@ __global__ void __maxnreg__(prom_regs<NPG>())
         const Unit un = decode_unit(u, args, BN);
         const uint32_t n = static_cast<uint32_t>(((un.nvalid + 15) / 16) * 16);
         const uint32_t idesc = make_idesc(FP8 ? 0u : 1u, n);
+        const int KPP = kpp_of(un);
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1u;
@@ -292,9 +337,10 @@ __global__ void __maxnreg__(prom_regs<NPG>())
       gph ^= 1u;
       return r;
     };
-    const int NP = (KB + KPP - 1) / KPP;  // promotions per tile
     for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
       const Unit un = decode_unit(u, args, BN);
+      const int KPP = kpp_of(un);
+      const int NP = (KB + KPP - 1) / KPP;  // promotions of this tile
       if (FP8) {
         // this tile's scales: activations [KB][BN] and the weight block scales
         if (!group_sync()) {  // the previous tile's readers are done
@@ -303,7 +349,11 @@ __global__ void __maxnreg__(prom_regs<NPG>())
         }
         for (int i = ptid; i < KB * BN; i += 128 * NPG) {
           const int kb = i / BN, j = i - kb * BN;
-          sa_s[i] = j < un.nvalid ? __ldg(args.act_scale + (size_t)(un.row0 + j) * KB + kb) : 0.f;
+          // the scales of the B row: the token's (gathered x) or the row's own (h)
+          const int r = j < un.nvalid ? (args.row_token ? __ldg(args.row_token + un.row0 + j)
+                                                         : un.row0 + j)
+                                      : -1;
+          sa_s[i] = r >= 0 ? __ldg(args.act_scale + (size_t)r * KB + kb) : 0.f;
         }
         // weight block scales [G][rows / 128][KB]: the tile's row of blocks
         // (DUAL: the two consecutive rows of its two tiles)
@@ -524,8 +574,11 @@ cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaSt
     a.out_scale = h->ws.hs;
     a.w_scale0 = h->w.gate_s;
     a.w_scale1 = h->w.up_s;
+    // short tiles gather the token rows (and scales) of the once-quantised
+    // x; taller ones read rows quantised into expert order by the dispatch
     a.act_scale = h->ws.xs;
-    const CUtensorMap& b = h->tm_xp[bi];
+    a.row_token = p.gather ? h->ws.row_token : nullptr;
+    const CUtensorMap& b = p.gather ? h->tm_xg : h->tm_xp[bi];
     const CUtensorMap &g = h->tm_gate, &u = h->tm_up;
     switch (p.bn) {
       case 16: return launch_one<16, true, true, 1>(h, g, u, b, a, s);
@@ -571,7 +624,7 @@ cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaSt
 // that the grid runs close to whole waves.
 cudaError_t launch_router_gemm(moe_handle* h, const void* x, int T, cudaStream_t s) {
   const Dims& dm = h->dims;
-  constexpr int BN = 128;
+  constexpr int BN = 256;  // tokens per tile: a 64-K stage holds 512 cycles of MMA work
   CUtensorMap tmx;
   {
     uint64_t dims[2] = {static_cast<uint64_t>(dm.d), static_cast<uint64_t>(T)};
@@ -591,14 +644,19 @@ cudaError_t launch_router_gemm(moe_handle* h, const void* x, int T, cudaStream_t
   a.k_blocks = 3 * dm.d / 64;
   a.ksplit = kTensorRouterSplits;
   a.split_stride = static_cast<size_t>(T) * dm.E;
+  // the high BF16 part is promoted every 128 K (its fp32 partial sums carry
+  // the logit's magnitude); the middle and low parts are 2^-8 and 2^-16 of
+  // it, so the tensor core's own accumulation over their whole slice adds
+  // error far below the 1e-5 band: one promotion per slice
   a.kpp = 2;
+  a.kpp_rest = a.k_blocks / kTensorRouterSplits;
   a.bn = BN;
   a.b_k = dm.d;
   a.m_valid = dm.E;
   a.out = h->ws.logits_part;
   a.ld = dm.E;
   a.status = h->ws.status;
-  return launch_one<BN, false, false, 2>(h, h->tm_router, h->tm_router, tmx, a, s);
+  return launch_one<BN, false, false, 4>(h, h->tm_router, h->tm_router, tmx, a, s);
 }
 
 }  // namespace smoe

@@ -34,7 +34,13 @@ struct GemmPlan {
   bool pair;    // BF16 on CTA pairs (2-SM MMA): units of 256 output features
   int m_tiles;  // output feature tiles (128 rows each, or 256 for a plain na = 2 unit)
   int k_blocks; // reduction / kernel K step
+  bool gather;  // gate/up: gather token rows from x with tile::gather4 (no row copies)
 };
+
+// Row tiles up to this height gather their B rows from x (a tile::gather4
+// moves four 128-byte rows, so taller tiles would be bound by TMA issue);
+// taller ones read rows the dispatch copied into expert order.
+constexpr int kGatherMaxBn = 32;
 
 struct Workspace {
   float* logits_part = nullptr;   // [splits][T][E]
@@ -48,8 +54,12 @@ struct Workspace {
   int32_t* unit_base = nullptr;   // [2][G+1] per-GEMM unit prefix
   int32_t* pair_row = nullptr;    // [T*k] row of each (token, slot)
   int32_t* row_token = nullptr;   // [Rmax] token of each row
-  void* xp = nullptr;             // [Rmax][d] gathered rows, BF16 or e4m3
-  float* xs = nullptr;            // [Rmax][d/128] FP8 activation scales
+  // B rows of the gate/up GEMM. Tall row tiles: [Rmax][d] gathered rows
+  // (BF16, or e4m3 with scales xs [Rmax][d/128]) in row order. Short row
+  // tiles gather from x itself; then, for FP8, rows [0, T) hold each
+  // token's quantised x once (scales likewise).
+  void* xp = nullptr;
+  float* xs = nullptr;
   void* hbuf = nullptr;           // [Rmax][f] SwiGLU output, BF16 or e4m3
   float* hs = nullptr;            // [Rmax][f/128] FP8 scales of h
   uint16_t* out = nullptr;        // [Rmax][d] BF16 per-row expert outputs
@@ -81,10 +91,13 @@ struct moe_handle {
   smoe::Dims dims{};
   smoe::Weights w;
   smoe::Workspace ws;
-  // TMA descriptors: weights (one per projection) and the two activation
-  // matrices, the latter once per row-tile height 16 * (i + 1), i < 16
+  // TMA descriptors: weights (one per projection); the gathered rows and h,
+  // once per row-tile height 16 * (i + 1), i < 16; and tm_xg, the
+  // one-row-box map short row tiles gather token rows through (over the
+  // quantised rows [0, T) of xp for FP8, made once; over the caller's x for
+  // BF16, made by each forward that gathers)
   CUtensorMap tm_gate, tm_up, tm_down, tm_router;
-  CUtensorMap tm_xp[16], tm_h[16];
+  CUtensorMap tm_xp[16], tm_h[16], tm_xg;
   int router_max_splits = 1;
   int64_t launches = 0;
   // options of the forward being launched: GEMM pipeline wait limit (0 =
@@ -139,7 +152,7 @@ GemmPlan plan_gate_up(const Dims& dm, int64_t T);
 GemmPlan plan_down(const Dims& dm, int64_t T);
 cudaError_t launch_route_scan(moe_handle* h, int T, const GemmPlan& p1, const GemmPlan& p2,
                               cudaStream_t s);
-cudaError_t launch_dispatch(moe_handle* h, const void* x, int T, cudaStream_t s);
+cudaError_t launch_dispatch(moe_handle* h, const void* x, int T, bool gather, cudaStream_t s);
 cudaError_t launch_combine(moe_handle* h, void* y, int T, cudaStream_t s);
 cudaError_t launch_act_quant(const void* x, int64_t rows, int d, uint8_t* q, float* s,
                              cudaStream_t st);
