@@ -106,6 +106,12 @@ typedef struct {
   int32_t weight_block_size[2];   /* {128, 128}; checked for the FP8 format */
   int32_t activation_scheme;      /* MOE_ACTIVATION_DYNAMIC */
   int64_t max_tokens;             /* largest T a forward will get; sizes the workspace */
+  /* Forwards of up to this many tokens (at most 128) run the whole layer as
+   * one cooperative launch when their row tiles are 16 rows: router, top-k,
+   * scan, placement, both GEMMs in one pipeline and the combine, separated by
+   * bounded grid barriers. 0 (the default of moe_config_init_k2): always the
+   * seven phase kernels. */
+  int64_t single_launch_max_tokens;
 } moe_config_t;
 
 /* Weights handed to moe_load_weights (caller-owned; copied by the call).
@@ -138,6 +144,12 @@ typedef struct {
  * forward runs on, so y holds no meaningful values. Nothing faults or hangs:
  * it is the path a real timeout takes. */
 #define MOE_FLAG_TEST_STALL 0x2u
+/* Run the layer as its seven phase kernels even where it would otherwise run
+ * as one launch (batches of up to 128 tokens whose row tiles are 16 rows:
+ * router, top-k, scan, placement, both GEMMs and the combine in one
+ * cooperative kernel). Both give the same routing; outputs agree within the
+ * tolerances (the logits are summed in another order). */
+#define MOE_FLAG_PHASE_KERNELS 0x4u
 
 typedef struct {
   int32_t* topk_ids_out;          /* optional device [T, k]: chosen experts, key-descending */

@@ -36,6 +36,7 @@ MOE_TOPK_NOAUX_TC = 0
 MOE_ACTIVATION_DYNAMIC = 0
 MOE_FLAG_SYNC_CHECK = 0x1
 MOE_FLAG_TEST_STALL = 0x2
+MOE_FLAG_PHASE_KERNELS = 0x4
 MOE_DEVICE_WAIT_TIMEOUT = 0x1
 MOE_DEVICE_BAD_EXPERT_ID = 0x2
 MOE_NUM_PHASES = 7
@@ -51,7 +52,7 @@ class moe_config_t(ctypes.Structure):
                 ("routed_scaling_factor", ctypes.c_float), ("scoring_func", ctypes.c_int32),
                 ("topk_method", ctypes.c_int32), ("weight_format", ctypes.c_int32),
                 ("weight_block_size", ctypes.c_int32 * 2), ("activation_scheme", ctypes.c_int32),
-                ("max_tokens", ctypes.c_int64)]
+                ("max_tokens", ctypes.c_int64), ("single_launch_max_tokens", ctypes.c_int64)]
 
 
 class moe_weights_t(ctypes.Structure):

@@ -159,6 +159,7 @@ moe_status_t validate(const moe_config_t* c, std::string* why) {
   const int64_t rows = c->max_tokens * (c->num_experts_per_tok + c->n_shared_experts);
   if (c->max_tokens > (1 << 20) || rows > (int64_t(1) << 30))
     return unsup("max_tokens too large (at most 2^20 tokens)");
+  if (c->single_launch_max_tokens < 0) return bad("single_launch_max_tokens must be >= 0");
   return MOE_OK;
 }
 
@@ -193,6 +194,8 @@ void free_all(moe_handle* h) {
   h->ev_in = h->ev_out = nullptr;
   for (cudaEvent_t e : h->prof_events) cudaEventDestroy(e);
   h->prof_events.clear();
+  if (h->prof_stamps) cudaFree(h->prof_stamps);
+  h->prof_stamps = nullptr;
 }
 
 }  // namespace
@@ -218,6 +221,7 @@ moe_status_t moe_config_init_k2(moe_config_t* c) {
   c->weight_block_size[1] = 128;
   c->activation_scheme = MOE_ACTIVATION_DYNAMIC;
   c->max_tokens = 8192;
+  c->single_launch_max_tokens = 0;
   return MOE_OK;
 }
 
@@ -287,13 +291,17 @@ moe_status_t moe_create(const moe_config_t* cfg, int device, moe_handle_t** out)
   A(&h->ws.logits_part, part_rows * E * 4, "router partials");
   A(&h->ws.ids, Tm * dm.k * 4, "ids");
   A(&h->ws.wts, Tm * dm.k * 4, "weights");
-  h->ws.zero_bytes = 256 + E * 4 + E * W * 4;
+  // zeroed at the start of every forward: [unit counters | counts | bitmaps |
+  // single-launch sync words]
+  h->ws.zero_bytes = 256 + E * 4 + E * W * 4 + (2 + G) * 4;
   {
     void* z = nullptr;
     A(&z, h->ws.zero_bytes, "counts/bitmap");
+    char* zc = static_cast<char*>(z);
     h->ws.sched = static_cast<int32_t*>(z);
-    h->ws.counts = z ? reinterpret_cast<int32_t*>(static_cast<char*>(z) + 256) : nullptr;
-    h->ws.bitmap = z ? reinterpret_cast<uint32_t*>(static_cast<char*>(z) + 256 + E * 4) : nullptr;
+    h->ws.counts = z ? reinterpret_cast<int32_t*>(zc + 256) : nullptr;
+    h->ws.bitmap = z ? reinterpret_cast<uint32_t*>(zc + 256 + E * 4) : nullptr;
+    h->ws.sync = z ? reinterpret_cast<uint32_t*>(zc + 256 + E * 4 + E * W * 4) : nullptr;
   }
   A(&h->ws.word_prefix, E * W * 4, "word prefix");
   A(&h->ws.offsets, (G + 1) * 4, "offsets");
@@ -485,7 +493,8 @@ moe_status_t moe_forward(moe_handle_t* h, const void* x, int64_t T, void* y,
     return fail(h, MOE_ERR_INVALID_ARG, "x and y overlap");
   if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 15)
     return fail(h, MOE_ERR_INVALID_ARG, "x and y must be 16-byte aligned");
-  if (opts && (opts->reserved != 0 || (opts->flags & ~(MOE_FLAG_SYNC_CHECK | MOE_FLAG_TEST_STALL))))
+  if (opts && (opts->reserved != 0 ||
+               (opts->flags & ~(MOE_FLAG_SYNC_CHECK | MOE_FLAG_TEST_STALL | MOE_FLAG_PHASE_KERNELS))))
     return fail(h, MOE_ERR_INVALID_ARG, "unknown option flags, or reserved != 0");
   DeviceGuard guard(h->device);
   if (!guard.ok) return fail(h, MOE_ERR_CUDA, "cudaSetDevice failed");
@@ -535,31 +544,73 @@ moe_status_t launch_forward(moe_handle* h, const void* x, int64_t T, void* y,
       return fail(h, MOE_ERR_CUDA, why);
   }
 
-  mark(0);
-  CUDA_TRY(h, cudaMemsetAsync(h->ws.sched, 0, h->ws.zero_bytes, s), "clear counts");
-  // without routed experts (a dense FFN layer) there is nothing to route: the
-  // router phases are empty and the shared groups take every token
-  const bool tensor_router = T >= smoe::kTensorRouterMinT;
-  if (dm.E > 0) {
-    if (tensor_router) {
-      CUDA_TRY(h, smoe::launch_router_gemm(h, x, Ti, s), "router GEMM launch");
-    } else {
-      CUDA_TRY(h, smoe::launch_router_logits(h, x, Ti, splits, s), "router logits launch");
+  const bool small = smoe::small_layer_supported(dm, T, h->cfg.single_launch_max_tokens) &&
+                     !(opts && (opts->flags & MOE_FLAG_PHASE_KERNELS));
+  if (small) {
+    // the whole layer in one cooperative launch; with profiling, its phase
+    // boundaries come from device timestamps
+    uint64_t* stamps = nullptr;
+    if (ev) {
+      stamps = h->prof_stamps + static_cast<size_t>(h->prof_next) * (MOE_NUM_PHASES + 1);
+      h->prof_small[h->prof_next] = 1;
     }
-  }
-  mark(1);
-  if (dm.E > 0) {
+    mark(0);
+    CUDA_TRY(h, cudaMemsetAsync(h->ws.sched, 0, h->ws.zero_bytes, s), "clear counts");
     CUDA_TRY(h,
-             smoe::launch_router_topk(h, Ti, tensor_router ? smoe::kTensorRouterSplits : splits,
-                                      forced, s, opts ? opts->topk_ids_out : nullptr,
+             smoe::launch_small_layer(h, x, Ti, y, forced, opts ? opts->topk_ids_out : nullptr,
                                       opts ? opts->topk_weights_out : nullptr,
-                                      opts ? opts->router_logits_out : nullptr),
-             "router top-k launch");
+                                      opts ? opts->router_logits_out : nullptr, stamps, s),
+             "single-launch layer");
+    for (int i = 1; i <= MOE_NUM_PHASES; ++i) mark(i);
+    if (ev) h->prof_next++;
+  } else {
+    if (ev) h->prof_small[h->prof_next] = 0;
+    mark(0);
+    CUDA_TRY(h, cudaMemsetAsync(h->ws.sched, 0, h->ws.zero_bytes, s), "clear counts");
+    // without routed experts (a dense FFN layer) there is nothing to route: the
+    // router phases are empty and the shared groups take every token
+    const bool tensor_router = T >= smoe::kTensorRouterMinT;
+    if (dm.E > 0) {
+      if (tensor_router) {
+        CUDA_TRY(h, smoe::launch_router_gemm(h, x, Ti, s), "router GEMM launch");
+      } else {
+        CUDA_TRY(h, smoe::launch_router_logits(h, x, Ti, splits, s), "router logits launch");
+      }
+    }
+    mark(1);
+    if (dm.E > 0) {
+      CUDA_TRY(h,
+               smoe::launch_router_topk(h, Ti, tensor_router ? smoe::kTensorRouterSplits : splits,
+                                        forced, s, opts ? opts->topk_ids_out : nullptr,
+                                        opts ? opts->topk_weights_out : nullptr,
+                                        opts ? opts->router_logits_out : nullptr),
+               "router top-k launch");
+    }
+    mark(2);
+    CUDA_TRY(h, smoe::launch_route_scan(h, Ti, p1, p2, s), "route scan launch");
+    mark(3);
+    CUDA_TRY(h, smoe::launch_dispatch(h, x, Ti, p1.gather, s), "dispatch launch");
+    mark(4);
+    if (dm.fp8) {
+      CUDA_TRY(h, smoe::launch_gemm_fp8(h, true, p1, s), "gate/up GEMM launch");
+    } else if (p1.pair) {
+      CUDA_TRY(h, smoe::launch_gemm_bf16_pair(h, true, p1, s), "gate/up GEMM launch");
+    } else {
+      CUDA_TRY(h, smoe::launch_gemm_bf16(h, true, p1, s), "gate/up GEMM launch");
+    }
+    mark(5);
+    if (dm.fp8) {
+      CUDA_TRY(h, smoe::launch_gemm_fp8(h, false, p2, s), "down GEMM launch");
+    } else if (p2.pair) {
+      CUDA_TRY(h, smoe::launch_gemm_bf16_pair(h, false, p2, s), "down GEMM launch");
+    } else {
+      CUDA_TRY(h, smoe::launch_gemm_bf16(h, false, p2, s), "down GEMM launch");
+    }
+    mark(6);
+    CUDA_TRY(h, smoe::launch_combine(h, y, Ti, s), "combine launch");
+    mark(7);
+    if (ev) h->prof_next++;
   }
-  mark(2);
-  CUDA_TRY(h, smoe::launch_route_scan(h, Ti, p1, p2, s), "route scan launch");
-  mark(3);
-  CUDA_TRY(h, smoe::launch_dispatch(h, x, Ti, p1.gather, s), "dispatch launch");
   if (opts && opts->expert_offsets_out && dm.E > 0)
     CUDA_TRY(h, cudaMemcpyAsync(opts->expert_offsets_out, h->ws.offsets, (dm.E + 1) * 4,
                                 cudaMemcpyDeviceToDevice, s),
@@ -568,26 +619,6 @@ moe_status_t launch_forward(moe_handle* h, const void* x, int64_t T, void* y,
     CUDA_TRY(h, cudaMemcpyAsync(opts->pair_rows_out, h->ws.pair_row, T * dm.k * 4,
                                 cudaMemcpyDeviceToDevice, s),
              "pair rows copy");
-  mark(4);
-  if (dm.fp8) {
-    CUDA_TRY(h, smoe::launch_gemm_fp8(h, true, p1, s), "gate/up GEMM launch");
-  } else if (p1.pair) {
-    CUDA_TRY(h, smoe::launch_gemm_bf16_pair(h, true, p1, s), "gate/up GEMM launch");
-  } else {
-    CUDA_TRY(h, smoe::launch_gemm_bf16(h, true, p1, s), "gate/up GEMM launch");
-  }
-  mark(5);
-  if (dm.fp8) {
-    CUDA_TRY(h, smoe::launch_gemm_fp8(h, false, p2, s), "down GEMM launch");
-  } else if (p2.pair) {
-    CUDA_TRY(h, smoe::launch_gemm_bf16_pair(h, false, p2, s), "down GEMM launch");
-  } else {
-    CUDA_TRY(h, smoe::launch_gemm_bf16(h, false, p2, s), "down GEMM launch");
-  }
-  mark(6);
-  CUDA_TRY(h, smoe::launch_combine(h, y, Ti, s), "combine launch");
-  mark(7);
-  if (ev) h->prof_next++;
 
   if (opts && (opts->flags & MOE_FLAG_SYNC_CHECK)) {
     uint32_t flags = 0;
@@ -722,7 +753,11 @@ moe_status_t moe_profile_enable(moe_handle_t* h, int32_t max_forwards) {
   h->prof_events.clear();
   h->prof_cap = 0;
   h->prof_next = 0;
+  if (h->prof_stamps) cudaFree(h->prof_stamps);
+  h->prof_stamps = nullptr;
   const size_t n = static_cast<size_t>(max_forwards) * (MOE_NUM_PHASES + 1);
+  if (n > 0) CUDA_TRY(h, cudaMalloc(&h->prof_stamps, n * 8), "profile stamps");
+  h->prof_small.assign(static_cast<size_t>(max_forwards), 0);
   h->prof_events.resize(n);
   for (size_t i = 0; i < n; ++i) {
     cudaError_t e = cudaEventCreate(&h->prof_events[i]);
@@ -744,11 +779,18 @@ moe_status_t moe_profile_read(moe_handle_t* h, float* ms, int32_t cap, int32_t* 
   for (int i = 0; i < n; ++i) {
     cudaEvent_t* ev = h->prof_events.data() + static_cast<size_t>(i) * (MOE_NUM_PHASES + 1);
     CUDA_TRY(h, cudaEventSynchronize(ev[MOE_NUM_PHASES]), "event sync");
+    uint64_t st[MOE_NUM_PHASES + 1] = {};
+    const bool small = h->prof_small[i] != 0;
+    if (small)
+      CUDA_TRY(h, cudaMemcpy(st, h->prof_stamps + static_cast<size_t>(i) * (MOE_NUM_PHASES + 1),
+                             sizeof st, cudaMemcpyDeviceToHost),
+               "stamps read");
     for (int p = 0; p < MOE_NUM_PHASES; ++p) {
       const int idx = i * MOE_NUM_PHASES + p;
       if (idx >= cap) return MOE_OK;
       float t = 0.f;
-      CUDA_TRY(h, cudaEventElapsedTime(&t, ev[p], ev[p + 1]), "event elapsed");
+      if (small) t = static_cast<float>(static_cast<double>(st[p + 1] - st[p]) * 1e-6);
+      else CUDA_TRY(h, cudaEventElapsedTime(&t, ev[p], ev[p + 1]), "event elapsed");
       ms[idx] = t;
     }
   }

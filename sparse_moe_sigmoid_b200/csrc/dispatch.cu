@@ -28,6 +28,7 @@
 #include <cuda_fp8.h>
 
 #include "internal.h"
+#include "route_common.cuh"
 
 namespace smoe {
 
@@ -108,42 +109,47 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* tmp, int* total)
   return incl - v;
 }
 
+// CTA 0 scans the per-group counts; CTAs 1.. compute, one warp per expert,
+// the running popcount of the expert's token bitmap over the words that can
+// hold tokens (ceil(T / 32) of the row's W).
 __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(
     const int32_t* __restrict__ counts, int E, int ns, int T, const uint32_t* __restrict__ bitmap,
     int W, int32_t* __restrict__ word_prefix, int32_t* __restrict__ offsets,
     int32_t* __restrict__ unit_base, int bn1, int mt1, int bn2, int mt2) {
-  __shared__ int tmp[kScanThreads];
-  const int G = E + ns;
-  const int g = threadIdx.x;  // G <= kMaxExperts + 8 < 1024
-  int c = 0;
-  if (g < E) c = counts[g];
-  else if (g < G) c = T;
-  const int u1 = mt1 * ((c + bn1 - 1) / bn1);
-  const int u2 = mt2 * ((c + bn2 - 1) / bn2);
-  int tot;
-  const int o = block_exclusive_scan(c, tmp, &tot);
-  if (g <= G) offsets[g] = o;
-  const int b1 = block_exclusive_scan(u1, tmp, &tot);
-  if (g <= G) unit_base[g] = b1;
-  const int b2 = block_exclusive_scan(u2, tmp, &tot);
-  if (g <= G) unit_base[(G + 1) + g] = b2;
-
-  // per-expert running popcount of the token bitmap
+  if (blockIdx.x == 0) {
+    __shared__ int tmp[kScanThreads];
+    const int G = E + ns;
+    const int g = threadIdx.x;  // G <= kMaxExperts + 16 < 1024
+    int c = 0;
+    if (g < E) c = counts[g];
+    else if (g < G) c = T;
+    const int u1 = mt1 * ((c + bn1 - 1) / bn1);
+    const int u2 = mt2 * ((c + bn2 - 1) / bn2);
+    int tot;
+    const int o = block_exclusive_scan(c, tmp, &tot);
+    if (g <= G) offsets[g] = o;
+    const int b1 = block_exclusive_scan(u1, tmp, &tot);
+    if (g <= G) unit_base[g] = b1;
+    const int b2 = block_exclusive_scan(u2, tmp, &tot);
+    if (g <= G) unit_base[(G + 1) + g] = b2;
+    return;
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int e = warp; e < E; e += kScanThreads / 32) {
-    int run = 0;
-    for (int w0 = 0; w0 < W; w0 += 32) {
-      const int w = w0 + lane;
-      const int v = w < W ? __popc(bitmap[(size_t)e * W + w]) : 0;
-      int incl = v;
+  const int e = (blockIdx.x - 1) * (kScanThreads / 32) + warp;
+  if (e >= E) return;
+  const int words = (T + 31) / 32;
+  int run = 0;
+  for (int w0 = 0; w0 < words; w0 += 32) {
+    const int w = w0 + lane;
+    const int v = w < words ? __popc(bitmap[(size_t)e * W + w]) : 0;
+    int incl = v;
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += n;
-      }
-      if (w < W) word_prefix[(size_t)e * W + w] = run + incl - v;
-      run += __shfl_sync(0xffffffffu, incl, 31);
+    for (int off = 1; off < 32; off <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += n;
     }
+    if (w < words) word_prefix[(size_t)e * W + w] = run + incl - v;
+    run += __shfl_sync(0xffffffffu, incl, 31);
   }
 }
 
@@ -151,77 +157,15 @@ cudaError_t launch_route_scan(moe_handle* h, int T, const GemmPlan& p1, const Ge
                               cudaStream_t s) {
   const Dims& dm = h->dims;
   const int W = static_cast<int>((dm.Tmax + 31) / 32);
-  route_scan_kernel<<<1, kScanThreads, 0, s>>>(h->ws.counts, dm.E, dm.ns, T, h->ws.bitmap, W,
-                                               h->ws.word_prefix, h->ws.offsets, h->ws.unit_base,
-                                               p1.bn, p1.m_tiles, p2.bn, p2.m_tiles);
+  const int blocks = 1 + (dm.E + kScanThreads / 32 - 1) / (kScanThreads / 32);
+  route_scan_kernel<<<blocks, kScanThreads, 0, s>>>(
+      h->ws.counts, dm.E, dm.ns, T, h->ws.bitmap, W, h->ws.word_prefix, h->ws.offsets,
+      h->ws.unit_base, p1.bn, p1.m_tiles, p2.bn, p2.m_tiles);
   h->launches++;
   return cudaGetLastError();
 }
 
 // ----------------------------------------------------------------- dispatch
-__device__ __forceinline__ int place_row(int i, int T, int k, int E, const int32_t* ids,
-                                         const uint32_t* bitmap, const int32_t* word_prefix,
-                                         const int32_t* offsets, int W, int* tok) {
-  const int nrouted = T * k;
-  if (i < nrouted) {
-    const int t = i / k;
-    const int e = ids[i];
-    const int w = t >> 5;
-    const uint32_t below = bitmap[(size_t)e * W + w] & ((1u << (t & 31)) - 1u);
-    *tok = t;
-    return offsets[e] + word_prefix[(size_t)e * W + w] + __popc(below);
-  }
-  const int s = (i - nrouted) / T;
-  const int t = (i - nrouted) % T;
-  *tok = t;
-  return offsets[E + s] + t;
-}
-
-// One row of d BF16 values -> d e4m3 codes + d/128 fp32 scales, by one warp:
-// each half-warp takes one 128-column group (16 lanes x 8 values).
-__device__ __forceinline__ void quant_row_e4m3(const __nv_bfloat16* __restrict__ src, int d,
-                                               uint8_t* __restrict__ dst,
-                                               float* __restrict__ scales, int lane) {
-  const int ngroups = d / 128;
-  for (int g0 = 0; g0 < ngroups; g0 += 2) {
-    const int gi = g0 + (lane >> 4);
-    const bool active = gi < ngroups;
-    const int col = gi * 128 + (lane & 15) * 8;
-    float v[8];
-    float amax = 0.f;
-    if (active) {
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src + col));
-      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f2 = __bfloat1622float2(p[j]);
-        v[2 * j] = f2.x;
-        v[2 * j + 1] = f2.y;
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
-    }
-#pragma unroll
-    for (int off = 8; off > 0; off >>= 1)
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    if (active) {
-      const float sa = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-      uint32_t packed[2];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float2 q;
-        q.x = __fdiv_rn(v[2 * j], sa);
-        q.y = __fdiv_rn(v[2 * j + 1], sa);
-        const __nv_fp8x2_storage_t b = __nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
-        if (j & 1) packed[j >> 1] |= static_cast<uint32_t>(b) << 16;
-        else packed[j >> 1] = static_cast<uint32_t>(b);
-      }
-      *reinterpret_cast<uint2*>(dst + col) = make_uint2(packed[0], packed[1]);
-      if ((lane & 15) == 0) scales[gi] = sa;
-    }
-  }
-}
-
 // Tall row tiles: one warp per row places the pair (pair_row, row_token)
 // and copies the token's x row into the gathered matrix in row order with
 // 16-byte loads and stores (FP8: quantises it on the way, as below).
@@ -242,8 +186,17 @@ __global__ void __launch_bounds__(256) dispatch_bf16_kernel(
   }
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
   uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)row * d);
-  const int n16 = d / 8;
-  for (int c = lane; c < n16; c += 32) dst[c] = __ldg(src + c);
+  const int n16 = d / 8;  // a multiple of 16 (d is a multiple of 128)
+  // four 16-byte loads in flight per lane before their stores
+  for (int c = lane; c < n16; c += 128) {
+    uint4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (c + 32 * j < n16) v[j] = __ldg(src + c + 32 * j);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (c + 32 * j < n16) dst[c + 32 * j] = v[j];
+  }
 }
 
 __global__ void __launch_bounds__(256) dispatch_fp8_kernel(
@@ -343,16 +296,6 @@ cudaError_t launch_dispatch(moe_handle* h, const void* x, int T, bool gather, cu
 // ------------------------------------------------------------------ combine
 // 8 columns per thread: one 16-byte load per expert row, one 16-byte store.
 constexpr int kCombineThreads = 128;
-
-__device__ __forceinline__ void add_row8(float (&acc)[8], const uint16_t* p, float w) {
-  const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
-  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {  // BF16 -> fp32 is exact: the bits move up by 16
-    acc[2 * i] = fmaf(w, __uint_as_float(u[i] << 16), acc[2 * i]);
-    acc[2 * i + 1] = fmaf(w, __uint_as_float(u[i] & 0xFFFF0000u), acc[2 * i + 1]);
-  }
-}
 
 __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const uint16_t* __restrict__ out, const int32_t* __restrict__ pair_row,

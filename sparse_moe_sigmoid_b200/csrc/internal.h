@@ -19,6 +19,7 @@ constexpr int kRouterTile = 64;   // router tile: 64 tokens x 64 experts
 constexpr int kRouterKTile = 32;
 constexpr int kRouterMaxSplits = 32;
 constexpr int kRouterGemvMaxT = 8;  // up to this many tokens the logits are a GEMV (one slice)
+constexpr int kSmallMaxT = 128;     // up to this many tokens the layer may run as one launch
 
 // Sizes derived from the config, fixed per handle.
 struct Dims {
@@ -64,6 +65,8 @@ struct Workspace {
   float* hs = nullptr;            // [Rmax][f/128] FP8 scales of h
   uint16_t* out = nullptr;        // [Rmax][d] BF16 per-row expert outputs
   uint32_t* status = nullptr;     // device status word
+  uint32_t* sync = nullptr;       // [2 + G] single-launch layer: grid barrier, abort, per-group
+                                  // finished gate/up warps (zeroed per forward)
   void* x_stage[2] = {};          // [Tmax][d] BF16 staging of the host entry points, used in turn
   void* y_stage[2] = {};          // [Tmax][d]
   size_t zero_bytes = 0;          // bytes of the sched+counts+bitmap region cleared per forward
@@ -108,6 +111,9 @@ struct moe_handle {
   // per-phase profiling
   std::vector<cudaEvent_t> prof_events;
   int prof_cap = 0, prof_next = 0;
+  // forwards run as one launch time their phases with device timestamps
+  uint64_t* prof_stamps = nullptr;  // [prof_cap][MOE_NUM_PHASES + 1] globaltimer ns
+  std::vector<char> prof_small;
   // host-memory entry points: upload and download streams, and per staging
   // buffer b the events "x uploaded", "forward done", "y downloaded"
   cudaStream_t up = nullptr, down = nullptr;
@@ -156,6 +162,11 @@ cudaError_t launch_dispatch(moe_handle* h, const void* x, int T, bool gather, cu
 cudaError_t launch_combine(moe_handle* h, void* y, int T, cudaStream_t s);
 cudaError_t launch_act_quant(const void* x, int64_t rows, int d, uint8_t* q, float* s,
                              cudaStream_t st);
+// layer_small.cu: the whole layer in one cooperative launch (16-row tiles)
+bool small_layer_supported(const Dims& dm, int64_t T, int64_t max_t);
+cudaError_t launch_small_layer(moe_handle* h, const void* x, int T, void* y,
+                               const int32_t* forced, int32_t* ids_out, float* wts_out,
+                               float* logits_out, uint64_t* stamps, cudaStream_t s);
 // gemm_bf16.cu / gemm_promoted.cu
 cudaError_t launch_gemm_bf16(moe_handle* h, bool gated, const GemmPlan& p, cudaStream_t s);
 cudaError_t launch_gemm_bf16_pair(moe_handle* h, bool gated, const GemmPlan& p, cudaStream_t s);

@@ -24,6 +24,7 @@
 #include <math.h>
 
 #include "internal.h"
+#include "route_common.cuh"
 
 namespace smoe {
 
@@ -129,197 +130,12 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const __nv_bfloat16*
   }
 }
 
-constexpr int kPerLane = kMaxExperts / 32;
-
-// Group-limited routing (n_group > 1; "Kimi K2 Base" raw config fields
-// n_group / topk_group, both 1 for K2, whose config post, §2.4, explains what
-// grouping is for). The experts form n_group contiguous groups of E / n_group;
-// a group scores the fp32 sum of its two largest keys (its one key for groups
-// of one); the topk_group best groups are kept, ties to the lower group; the
-// other groups' keys become -inf so that the top-k below never picks them.
-// One warp: the keys go through this warp's shared-memory row, lane g < n_group
-// scans group g, and the groups are picked by topk_group shuffle arg-max rounds.
-__device__ __forceinline__ void group_filter(float (&key)[kMaxExperts / 32], int E, int n_group,
-                                             int topk_group, float* __restrict__ row,
-                                             int lane) {
-  const unsigned full = 0xffffffffu;
-#pragma unroll
-  for (int i = 0; i < kMaxExperts / 32; ++i)
-    if (lane + 32 * i < E) row[lane + 32 * i] = key[i];
-  __syncwarp();
-  const int gs = E / n_group;
-  float gscore = -INFINITY;
-  if (lane < n_group) {
-    float b1 = -INFINITY, b2 = -INFINITY;  // the two largest keys of group `lane`
-    for (int j = 0; j < gs; ++j) {
-      const float v = row[lane * gs + j];
-      if (v > b1) {
-        b2 = b1;
-        b1 = v;
-      } else if (v > b2) {
-        b2 = v;
-      }
-    }
-    gscore = gs >= 2 ? b1 + b2 : b1;
-  }
-  uint32_t kept = 0;  // bit g: group g kept
-  for (int r = 0; r < topk_group; ++r) {
-    float bv = (lane < n_group && !((kept >> lane) & 1u)) ? gscore : -INFINITY;
-    int bi = (lane < n_group && !((kept >> lane) & 1u)) ? lane : 0x7fffffff;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(full, bv, off);
-      const int oi = __shfl_xor_sync(full, bi, off);
-      if (ov > bv || (ov == bv && oi < bi)) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    if (bi >= n_group) {  // NaN or -inf scores only: the lowest group not yet kept
-      bi = 0;
-      while (bi < n_group && ((kept >> bi) & 1u)) ++bi;
-    }
-    kept |= 1u << bi;
-  }
-#pragma unroll
-  for (int i = 0; i < kMaxExperts / 32; ++i) {
-    const int e = lane + 32 * i;
-    if (e < E && !((kept >> (e / gs)) & 1u)) key[i] = -INFINITY;
-  }
-  __syncwarp();
-}
-
-__global__ void __launch_bounds__(256) router_topk_kernel(
-    const float* __restrict__ part, int splits, const float* __restrict__ bias, int T, int E,
-    int k, float scale, int norm, const int32_t* __restrict__ forced, int32_t* __restrict__ ids,
-    float* __restrict__ wts, int32_t* __restrict__ counts, uint32_t* __restrict__ bitmap,
-    int W, uint32_t* __restrict__ status, int32_t* __restrict__ ids_out,
-    float* __restrict__ wts_out, float* __restrict__ logits_out, int n_group, int topk_group) {
+__global__ void __launch_bounds__(256) router_topk_kernel(TopkArgs a) {
   __shared__ float group_rows[256 / 32][kMaxExperts];  // one key row per warp (group filter)
   const int lane = threadIdx.x & 31;
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (t >= T) return;
-  const unsigned full = 0xffffffffu;
-
-  float key[kPerLane], sc[kPerLane], lg[kPerLane];
-#pragma unroll
-  for (int i = 0; i < kPerLane; ++i) lg[i] = 0.f;
-  // slices in order (a deterministic sum); the loads of a slice's experts are
-  // independent, so they are issued together, four slices at a time
-#pragma unroll 4
-  for (int s = 0; s < splits; ++s) {
-    const float* ps = part + ((size_t)s * T + t) * E;
-    float v[kPerLane];
-#pragma unroll
-    for (int i = 0; i < kPerLane; ++i) v[i] = lane + 32 * i < E ? __ldg(ps + lane + 32 * i) : 0.f;
-#pragma unroll
-    for (int i = 0; i < kPerLane; ++i) lg[i] += v[i];
-  }
-#pragma unroll
-  for (int i = 0; i < kPerLane; ++i) {
-    const int e = lane + 32 * i;
-    if (e < E) {
-      const float l = lg[i];
-      if (logits_out) logits_out[(size_t)t * E + e] = l;
-      const float p = 1.f / (1.f + expf(-l));
-      sc[i] = p;
-      key[i] = p + bias[e];
-    } else {
-      sc[i] = 0.f;
-      key[i] = -INFINITY;
-    }
-  }
-
-  int my_id = 0;
-  float my_sc = 0.f;
-  bool use_forced = forced != nullptr;
-  if (use_forced) {
-    int e = -1;
-    if (lane < k) e = forced[(size_t)t * k + lane];
-    bool bad = lane < k && (e < 0 || e >= E);
-    for (int jj = 0; jj < k; ++jj) {
-      const int other = __shfl_sync(full, e, jj);
-      if (lane < k && jj < lane && other == e) bad = true;
-    }
-    if (__any_sync(full, bad)) {
-      // an out-of-range or repeated id: report it and select normally, which
-      // keeps the dispatch's bookkeeping consistent
-      if (lane == 0) atomicOr(status, MOE_DEVICE_BAD_EXPERT_ID);
-      use_forced = false;
-    } else {
-      // each lane j < k fetches its expert's score from the owning lane
-      for (int jj = 0; jj < k; ++jj) {
-        const int ej = __shfl_sync(full, e, jj);
-        float v = 0.f;
-#pragma unroll
-        for (int i = 0; i < kPerLane; ++i)
-          if (i == (ej >> 5)) v = sc[i];
-        v = __shfl_sync(full, v, ej & 31);
-        if (lane == jj) {
-          my_id = ej;
-          my_sc = v;
-        }
-      }
-    }
-  }
-  if (!use_forced) {
-    if (n_group > 1) group_filter(key, E, n_group, topk_group, group_rows[threadIdx.x >> 5], lane);
-    uint32_t taken = 0;  // bit i: expert lane + 32 i already chosen
-    for (int j = 0; j < k; ++j) {
-      float bk = -INFINITY;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int i = 0; i < kPerLane; ++i) {
-        const int e = lane + 32 * i;
-        if (e < E && !((taken >> i) & 1u) && (key[i] > bk || (key[i] == bk && e < bi))) {
-          bk = key[i];
-          bi = e;
-        }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ok = __shfl_xor_sync(full, bk, off);
-        const int oi = __shfl_xor_sync(full, bi, off);
-        if (ok > bk || (ok == bk && oi < bi)) {
-          bk = ok;
-          bi = oi;
-        }
-      }
-      if (bi >= E) {  // NaN keys: nothing comparable left; keep the bookkeeping valid
-        if (lane == 0) atomicOr(status, MOE_DEVICE_BAD_EXPERT_ID);
-        bi = 0;
-        while (bi < E) {  // smallest id not yet taken
-          const int owner = bi & 31;
-          const uint32_t tk = __shfl_sync(full, taken, owner);
-          if (!((tk >> (bi >> 5)) & 1u)) break;
-          ++bi;
-        }
-      }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      float v = 0.f;
-#pragma unroll
-      for (int i = 0; i < kPerLane; ++i)
-        if (i == (bi >> 5)) v = sc[i];
-      v = __shfl_sync(full, v, bi & 31);
-      if (lane == j) {
-        my_id = bi;
-        my_sc = v;
-      }
-    }
-  }
-
-  float total = lane < k ? my_sc : 0.f;
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) total += __shfl_xor_sync(full, total, off);
-  if (lane < k) {
-    const float w = norm ? my_sc / total * scale : my_sc * scale;
-    ids[(size_t)t * k + lane] = my_id;
-    wts[(size_t)t * k + lane] = w;
-    if (ids_out) ids_out[(size_t)t * k + lane] = my_id;
-    if (wts_out) wts_out[(size_t)t * k + lane] = w;
-    atomicAdd(&counts[my_id], 1);
-    atomicOr(&bitmap[(size_t)my_id * W + (t >> 5)], 1u << (t & 31));
-  }
+  if (t >= a.T) return;
+  route_token(a, t, group_rows[threadIdx.x >> 5], lane);
 }
 
 // Few tokens (T <= kRouterGemvMaxT): the 64 x 64 tiles of router_logits_kernel
@@ -391,10 +207,11 @@ cudaError_t launch_router_topk(moe_handle* h, int T, int splits, const int32_t* 
   const Dims& dm = h->dims;
   const int W = static_cast<int>((dm.Tmax + 31) / 32);
   const int blocks = (T * 32 + 255) / 256;
-  router_topk_kernel<<<blocks, 256, 0, s>>>(
-      h->ws.logits_part, splits, h->w.bias, T, dm.E, dm.k, h->cfg.routed_scaling_factor,
-      h->cfg.norm_topk_prob, forced, h->ws.ids, h->ws.wts, h->ws.counts, h->ws.bitmap, W,
-      h->ws.status, ids_out, wts_out, logits_out, h->cfg.n_group, h->cfg.topk_group);
+  const TopkArgs a{h->ws.logits_part, splits, h->w.bias, T, dm.E, dm.k,
+                   h->cfg.routed_scaling_factor, h->cfg.norm_topk_prob, forced, h->ws.ids,
+                   h->ws.wts, h->ws.counts, h->ws.bitmap, W, h->ws.status, ids_out, wts_out,
+                   logits_out, h->cfg.n_group, h->cfg.topk_group};
+  router_topk_kernel<<<blocks, 256, 0, s>>>(a);
   h->launches++;
   return cudaGetLastError();
 }
@@ -414,9 +231,9 @@ cudaError_t launch_router_raw(const void* x, const float* router_weight, const f
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int blocks = (T * 32 + 255) / 256;
-  router_topk_kernel<<<blocks, 256, 0, s>>>(part, splits, bias, T, E, k, scale, norm, nullptr, ids,
-                                            wts, counts, bitmap, W, status, nullptr, nullptr,
-                                            nullptr, 1, 1);
+  const TopkArgs a{part, splits, bias, T, E, k, scale, norm, nullptr, ids, wts, counts, bitmap,
+                   W, status, nullptr, nullptr, nullptr, 1, 1};
+  router_topk_kernel<<<blocks, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 

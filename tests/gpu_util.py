@@ -75,7 +75,8 @@ def make_layer(shape, T, fmt="bf16", seed=synth.SEED, device="cuda", identical=F
     return Layer(shape, fmt, x, Wg, b, ew)
 
 
-def create_handle(smoe, layer: Layer, max_tokens: int, device: int = 0):
+def create_handle(smoe, layer: Layer, max_tokens: int, device: int = 0,
+                  single_launch_max_tokens: int = 0):
     s = layer.shape
     cfg = smoe.moe_config_init_k2(
         hidden_size=s.hidden_size, moe_intermediate_size=s.moe_intermediate_size,
@@ -83,6 +84,7 @@ def create_handle(smoe, layer: Layer, max_tokens: int, device: int = 0):
         n_shared_experts=s.n_shared_experts, routed_scaling_factor=s.routed_scaling_factor,
         norm_topk_prob=int(s.norm_topk_prob), max_tokens=max_tokens,
         n_group=s.n_group, topk_group=s.topk_group,
+        single_launch_max_tokens=single_launch_max_tokens,
         weight_format=smoe.MOE_WEIGHT_BF16 if layer.fmt == "bf16" else smoe.MOE_WEIGHT_FP8_E4M3_BLOCK)
     h = smoe.moe_create(cfg, device)
     ew = layer.ew
@@ -109,7 +111,7 @@ class Run:
 
 
 def run(smoe, h, layer: Layer, x: Optional[torch.Tensor] = None, forced=None,
-        permutation: bool = False) -> Run:
+        permutation: bool = False, flags: int = 0) -> Run:
     x = layer.x if x is None else x
     T, k, E = x.shape[0], layer.shape.num_experts_per_tok, layer.shape.n_routed_experts
     y = torch.empty_like(x)
@@ -120,7 +122,8 @@ def run(smoe, h, layer: Layer, x: Optional[torch.Tensor] = None, forced=None,
         off = torch.full((E + 1,), -1, dtype=torch.int32, device=x.device)
         pr = torch.full((T, k), -1, dtype=torch.int32, device=x.device)
     smoe.moe_forward(h, x, y, topk_ids_out=ids, topk_weights_out=w, forced_topk_ids=forced,
-                     flags=smoe.MOE_FLAG_SYNC_CHECK, expert_offsets_out=off, pair_rows_out=pr)
+                     flags=smoe.MOE_FLAG_SYNC_CHECK | flags, expert_offsets_out=off,
+                     pair_rows_out=pr)
     return Run(y, ids, w, off, pr)
 
 

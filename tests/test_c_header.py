@@ -28,9 +28,9 @@ int main(void) {
   if (moe_create(&c, 0, &h) != MOE_ERR_UNSUPPORTED || h != NULL) return 4;
   if (strcmp(moe_status_string(MOE_OK), "ok") != 0) return 5;
   if (moe_forward(NULL, NULL, 0, NULL, NULL, NULL) != MOE_ERR_INVALID_ARG) return 6;
-  printf("config %zu %zu %zu %zu\n", sizeof(moe_config_t),
+  printf("config %zu %zu %zu %zu %zu\n", sizeof(moe_config_t),
          offsetof(moe_config_t, routed_scaling_factor), offsetof(moe_config_t, weight_block_size),
-         offsetof(moe_config_t, max_tokens));
+         offsetof(moe_config_t, max_tokens), offsetof(moe_config_t, single_launch_max_tokens));
   printf("weights %zu %zu\n", sizeof(moe_weights_t), offsetof(moe_weights_t, shared_down_scale));
   printf("opts %zu %zu %zu %zu\n", sizeof(moe_forward_opts_t), offsetof(moe_forward_opts_t, flags),
          offsetof(moe_forward_opts_t, pair_rows_out), offsetof(moe_forward_opts_t, wait_limit_ns));
@@ -63,7 +63,8 @@ def test_header_is_c99_and_layouts_match_the_binding(smoe, tmp_path):
     got = {line.split()[0]: [int(v) for v in line.split()[1:]] for line in r.stdout.splitlines()}
     C, W, O = smoe.moe_config_t, smoe.moe_weights_t, smoe.moe_forward_opts_t
     assert got["config"] == [ctypes.sizeof(C), C.routed_scaling_factor.offset,
-                             C.weight_block_size.offset, C.max_tokens.offset]
+                             C.weight_block_size.offset, C.max_tokens.offset,
+                             C.single_launch_max_tokens.offset]
     assert got["weights"] == [ctypes.sizeof(W), W.shared_down_scale.offset]
     assert got["opts"] == [ctypes.sizeof(O), O.flags.offset, O.pair_rows_out.offset,
                            O.wait_limit_ns.offset]
