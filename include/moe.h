@@ -261,6 +261,23 @@ moe_status_t moe_profile_read(moe_handle_t* h, float* ms, int32_t cap, int32_t* 
 moe_status_t moe_act_quant_e4m3(const void* x, int64_t rows, int32_t cols, void* q,
                                 float* scales, void* stream);
 
+/* The layer's output from per-pair expert outputs already in (token, slot)
+ * order: y[t] = sum_j weights[t, j] * pair_out[t * k + j] + shared_out[t],
+ * summed in fp32 in slot order and rounded once to BF16 (the output
+ * y[t] = sum_j w[t,j] E_{id[t,j]}(x_t) + S(x_t) of the layer above). It is
+ * the last step of an expert-parallel forward, after each pair's output has
+ * come back from the GPU that owns its expert ("Behind Kimi-K2's Config"
+ * §2.1: EP across GPUs).
+ *   pair_out    device BF16 [T * k, hidden_size], 16-byte aligned
+ *   weights     device fp32 [T, k]
+ *   shared_out  device BF16 [T, hidden_size], 16-byte aligned, or NULL
+ *   y           device BF16 [T, hidden_size] (written), 16-byte aligned
+ * hidden_size a multiple of 8, 1 <= k <= 32, else MOE_ERR_INVALID_ARG. No
+ * handle: runs on the current device, asynchronous on `stream`. */
+moe_status_t moe_combine_rows(const void* pair_out, const float* weights, const void* shared_out,
+                              int64_t T, int32_t hidden_size, int32_t num_experts_per_tok,
+                              void* y, void* stream);
+
 /* Number of kernels this handle has launched so far. */
 int64_t moe_launch_count(const moe_handle_t* h);
 

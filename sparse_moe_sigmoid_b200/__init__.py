@@ -93,6 +93,8 @@ _sig = {
                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "moe_act_quant_e4m3": (_S, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p,
                                 ctypes.c_void_p, ctypes.c_void_p]),
+    "moe_combine_rows": (_S, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                              ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]),
     "moe_launch_count": (ctypes.c_int64, [_H]),
     "moe_destroy": (None, [_H]),
     "moe_status_string": (ctypes.c_char_p, [_S]),
@@ -259,6 +261,15 @@ def moe_act_quant_e4m3(x, q, scales, stream=None):
     rows, cols = x.shape
     st = _lib.moe_act_quant_e4m3(_ptr(x), rows, cols, _ptr(q), _ptr(scales), _stream(stream))
     _check(st, "moe_act_quant_e4m3")
+
+
+def moe_combine_rows(pair_out, weights, shared_out, y, stream=None):
+    """y[t] = sum_j weights[t, j] * pair_out[t * k + j] + shared_out[t] (BF16
+    rows in (token, slot) order; shared_out may be None)."""
+    T, k = weights.shape
+    st = _lib.moe_combine_rows(_ptr(pair_out), _ptr(weights), _ptr(shared_out), T,
+                               pair_out.shape[1], k, _ptr(y), _stream(stream))
+    _check(st, "moe_combine_rows")
 
 
 def moe_launch_count(h) -> int:

@@ -810,6 +810,24 @@ moe_status_t moe_act_quant_e4m3(const void* x, int64_t rows, int32_t cols, void*
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+moe_status_t moe_combine_rows(const void* pair_out, const float* weights, const void* shared_out,
+                              int64_t T, int32_t hidden_size, int32_t num_experts_per_tok,
+                              void* y, void* stream) {
+  if (T < 0 || hidden_size <= 0 || hidden_size % 8 || num_experts_per_tok <= 0 ||
+      num_experts_per_tok > smoe::kMaxTopK)
+    return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (pair_out == nullptr || weights == nullptr || y == nullptr) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(pair_out) | reinterpret_cast<uintptr_t>(shared_out) |
+       reinterpret_cast<uintptr_t>(y)) & 15)
+    return MOE_ERR_INVALID_ARG;
+  if (T > (int64_t(1) << 31) - 1) return MOE_ERR_INVALID_ARG;
+  cudaError_t e = smoe::launch_combine_rows(pair_out, weights, shared_out, static_cast<int>(T),
+                                            hidden_size, num_experts_per_tok, y,
+                                            static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 int64_t moe_launch_count(const moe_handle_t* h) { return h ? h->launches : 0; }
 
 void moe_destroy(moe_handle_t* h) {

@@ -48,6 +48,12 @@ static int pick_bn(double want, const int* cands, int n) {
 #ifndef SMOE_BN_FACTOR
 #define SMOE_BN_FACTOR 3.0  // tuning constant
 #endif
+// FP8 gate/up tiles up to this height gather their token rows from the
+// once-quantised x (taller FP8 tiles are bound by the promotion, not by TMA
+// issue, so gathering may pay there too: a tuning constant)
+#ifndef SMOE_FP8_GATHER_MAX_BN
+#define SMOE_FP8_GATHER_MAX_BN 32
+#endif
 // mean rows per routed expert (T k / E); every token's row in each shared
 // group when there are no routed experts
 static double rows_per_group(const Dims& dm, int64_t T) {
@@ -62,7 +68,7 @@ GemmPlan plan_gate_up(const Dims& dm, int64_t T) {
   p.bn = dm.fp8 ? pick_bn(want, fp8_bn, 4) : pick_bn(want, bf16_bn, 9);
   p.na = 2;
   p.pair = !dm.fp8 && pair_bn_supported(p.bn) && dm.f % 256 == 0;
-  p.gather = !p.pair && p.bn <= kGatherMaxBn;
+  p.gather = !p.pair && p.bn <= (dm.fp8 ? SMOE_FP8_GATHER_MAX_BN : kGatherMaxBn);
   p.m_tiles = dm.f / (p.pair ? 256 : kBlock);
   p.k_blocks = dm.fp8 ? dm.d / 128 : dm.d / 64;
   return p;
@@ -328,6 +334,41 @@ cudaError_t launch_combine(moe_handle* h, void* y, int T, cudaStream_t s) {
                                                   h->ws.offsets, T, dm.d, dm.k, dm.E, dm.ns,
                                                   static_cast<__nv_bfloat16*>(y));
   h->launches++;
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------- combine of rows
+// The combine step on rows already in (token, slot) order: the last step of
+// an expert-parallel forward, after each pair's output came back from the
+// rank that owns its expert. Same arithmetic as combine_kernel.
+__global__ void __launch_bounds__(kCombineThreads)
+    combine_rows_kernel(const uint16_t* __restrict__ pair_out, const float* __restrict__ wts,
+                        const uint16_t* __restrict__ shared, int T, int d, int k,
+                        __nv_bfloat16* __restrict__ y) {
+  const int t = blockIdx.x;
+  const int c = (blockIdx.y * blockDim.x + threadIdx.x) * 8;
+  if (c >= d) return;
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  for (int j = 0; j < k; ++j)
+    add_row8(acc, pair_out + ((size_t)t * k + j) * d + c, wts[(size_t)t * k + j]);
+  if (shared) add_row8(acc, shared + (size_t)t * d + c, 1.f);
+  uint32_t pk[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+    pk[i] = *reinterpret_cast<uint32_t*>(&b);
+  }
+  *reinterpret_cast<uint4*>(y + (size_t)t * d + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+}
+
+cudaError_t launch_combine_rows(const void* pair_out, const float* wts, const void* shared, int T,
+                                int d, int k, void* y, cudaStream_t s) {
+  dim3 grid(T, (d / 8 + kCombineThreads - 1) / kCombineThreads);
+  combine_rows_kernel<<<grid, kCombineThreads, 0, s>>>(
+      static_cast<const uint16_t*>(pair_out), wts, static_cast<const uint16_t*>(shared), T, d, k,
+      static_cast<__nv_bfloat16*>(y));
   return cudaGetLastError();
 }
 

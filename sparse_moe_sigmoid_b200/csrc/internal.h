@@ -160,6 +160,8 @@ cudaError_t launch_route_scan(moe_handle* h, int T, const GemmPlan& p1, const Ge
                               cudaStream_t s);
 cudaError_t launch_dispatch(moe_handle* h, const void* x, int T, bool gather, cudaStream_t s);
 cudaError_t launch_combine(moe_handle* h, void* y, int T, cudaStream_t s);
+cudaError_t launch_combine_rows(const void* pair_out, const float* wts, const void* shared, int T,
+                                int d, int k, void* y, cudaStream_t s);
 cudaError_t launch_act_quant(const void* x, int64_t rows, int d, uint8_t* q, float* s,
                              cudaStream_t st);
 // layer_small.cu: the whole layer in one cooperative launch (16-row tiles)
