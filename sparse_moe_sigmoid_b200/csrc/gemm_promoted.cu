@@ -88,8 +88,16 @@ struct PromCfg {
   static_assert(kPBufs >= 2, "the promotion needs two partial buffers at least");
   static_assert(FP8 || !GATED, "the BF16 promoted GEMM is plain");
   static_assert(!GATED || BN <= 128, "a gathered tile takes at most one gather4 per lane");
-  // scale staging of FP8: activation scales [KB][BN] and weight scales [2][KB]
-  static constexpr int scale_bytes(int kb) { return FP8 ? (kb * BN + 2 * kb) * 4 : 0; }
+  // Tall tiles (three promotion warpgroups, the promotion-bound regime) stage
+  // the products s_w * s_x per block and row, once per tile, so the promotion
+  // does one multiply-add per value; the others stage s_x and s_w and
+  // multiply per value (one stage more of the ring at mid sizes).
+  static constexpr bool kPreMul = FP8 && NPG >= 3;
+  // scale staging of FP8: [KB][BN] activation scales (or products, one array
+  // per weight tile) and [2][KB] weight scales
+  static constexpr int scale_bytes(int kb) {
+    return !FP8 ? 0 : kPreMul ? (kTwoA ? 2 : 1) * kb * BN * 4 : (kb * BN + 2 * kb) * 4;
+  }
   static constexpr int stages(int kb) {
     const int n = (kPromSmemBudget - kBarrierBytes - scale_bytes(kb) - kAmaxBytes) / kStage;
     return n > kPromMaxStages ? kPromMaxStages : n;
@@ -148,8 +156,10 @@ __global__ void __maxnreg__(prom_regs<NPG>())
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   float* sa_s = reinterpret_cast<float*>(smem + S * C::kStage);  // [KB][BN] (FP8)
-  float* sw_s = sa_s + (FP8 ? KB * BN : 0);                       // [2][KB] (FP8)
-  float* amax_s = sw_s + (FP8 ? 2 * KB : 0);                      // [4][BN] (gated)
+  // kPreMul: sa_s holds s_w0 * s_x and sb_s s_w1 * s_x; else sw_s the s_w
+  float* sb_s = sa_s + (C::kPreMul && C::kTwoA ? KB * BN : 0);
+  float* sw_s = sa_s + (FP8 ? (C::kPreMul ? (C::kTwoA ? 2 : 1) * KB * BN : KB * BN) : 0);
+  float* amax_s = sw_s + (FP8 && !C::kPreMul ? 2 * KB : 0);       // [4][BN] (gated)
   uint64_t* full = reinterpret_cast<uint64_t*>(
       (reinterpret_cast<uintptr_t>(amax_s + (GATED ? 4 * BN : 0)) + 7) & ~uintptr_t(7));
   uint64_t* empty = full + kPromMaxStages;
@@ -347,22 +357,30 @@ __global__ void __maxnreg__(prom_regs<NPG>())
           ok = false;
           break;
         }
+        // weight block scales [G][rows / 128][KB]: the tile's row of blocks
+        // (DUAL: the two consecutive rows of its two tiles)
+        const size_t wrow = DUAL ? ((size_t)un.g * 2 * args.m_tiles + 2 * un.mt) * KB
+                                 : ((size_t)un.g * args.m_tiles + un.mt) * KB;
+        const float* ws1 = GATED ? args.w_scale1 + wrow : args.w_scale0 + wrow + KB;
         for (int i = ptid; i < KB * BN; i += 128 * NPG) {
           const int kb = i / BN, j = i - kb * BN;
           // the scales of the B row: the token's (gathered x) or the row's own (h)
           const int r = j < un.nvalid ? (args.row_token ? __ldg(args.row_token + un.row0 + j)
                                                          : un.row0 + j)
                                       : -1;
-          sa_s[i] = r >= 0 ? __ldg(args.act_scale + (size_t)r * KB + kb) : 0.f;
+          const float sx = r >= 0 ? __ldg(args.act_scale + (size_t)r * KB + kb) : 0.f;
+          if (C::kPreMul) {  // the products the promotion multiplies by
+            sa_s[i] = __ldg(args.w_scale0 + wrow + kb) * sx;
+            if (C::kTwoA) sb_s[i] = __ldg(ws1 + kb) * sx;
+          } else {
+            sa_s[i] = sx;
+          }
         }
-        // weight block scales [G][rows / 128][KB]: the tile's row of blocks
-        // (DUAL: the two consecutive rows of its two tiles)
-        const size_t wrow = DUAL ? ((size_t)un.g * 2 * args.m_tiles + 2 * un.mt) * KB
-                                 : ((size_t)un.g * args.m_tiles + un.mt) * KB;
-        for (int i = ptid; i < KB; i += 128 * NPG) {
-          sw_s[i] = __ldg(args.w_scale0 + wrow + i);
-          if (GATED) sw_s[KB + i] = __ldg(args.w_scale1 + wrow + i);
-          if (DUAL) sw_s[KB + i] = __ldg(args.w_scale0 + wrow + KB + i);
+        if (!C::kPreMul) {
+          for (int i = ptid; i < KB; i += 128 * NPG) {
+            sw_s[i] = __ldg(args.w_scale0 + wrow + i);
+            if (C::kTwoA) sw_s[KB + i] = __ldg(ws1 + i);
+          }
         }
         if (!group_sync()) {
           ok = false;
@@ -384,9 +402,10 @@ __global__ void __maxnreg__(prom_regs<NPG>())
           break;
         }
         tc_fence_after();
-        const float sw0 = FP8 ? sw_s[pg] : 1.f;
-        const float sw1 = (FP8 && C::kTwoA) ? sw_s[KB + pg] : 0.f;
+        const float sw0 = FP8 && !C::kPreMul ? sw_s[pg] : 1.f;
+        const float sw1 = (FP8 && C::kTwoA && !C::kPreMul) ? sw_s[KB + pg] : 0.f;
         const float* sa = sa_s + pg * BN + c_begin;
+        const float* sb = sb_s + pg * BN + c_begin;
         // loads in batches of kBatch columns, one wait per batch, then the
         // arithmetic: tcgen05.wait::ld waits for all outstanding loads, so a
         // wait per 16-column chunk would pay the TMEM round trip once per
@@ -416,17 +435,27 @@ __global__ void __maxnreg__(prom_regs<NPG>())
                 for (int jj = c * 16; jj < c * 16 + 16; jj += 4) {
                   const int j = b0 + jj;
                   const float4 s4 = *reinterpret_cast<const float4*>(sa + j);
-                  float c00, c01, c02, c03;
-                  mul2(c00, c01, sw0, sw0, s4.x, s4.y);
-                  mul2(c02, c03, sw0, sw0, s4.z, s4.w);
+                  float c00 = s4.x, c01 = s4.y, c02 = s4.z, c03 = s4.w;
+                  if (!C::kPreMul) {
+                    mul2(c00, c01, sw0, sw0, s4.x, s4.y);
+                    mul2(c02, c03, sw0, sw0, s4.z, s4.w);
+                  }
                   fma2(acc0[j], acc0[j + 1], __uint_as_float(g[jj]), __uint_as_float(g[jj + 1]),
                        c00, c01);
                   fma2(acc0[j + 2], acc0[j + 3], __uint_as_float(g[jj + 2]),
                        __uint_as_float(g[jj + 3]), c02, c03);
                   if (C::kTwoA) {
                     float c10, c11, c12, c13;
-                    mul2(c10, c11, sw1, sw1, s4.x, s4.y);
-                    mul2(c12, c13, sw1, sw1, s4.z, s4.w);
+                    if (C::kPreMul) {
+                      const float4 t4 = *reinterpret_cast<const float4*>(sb + j);
+                      c10 = t4.x;
+                      c11 = t4.y;
+                      c12 = t4.z;
+                      c13 = t4.w;
+                    } else {
+                      mul2(c10, c11, sw1, sw1, s4.x, s4.y);
+                      mul2(c12, c13, sw1, sw1, s4.z, s4.w);
+                    }
                     fma2(acc1[j], acc1[j + 1], __uint_as_float(v[jj]), __uint_as_float(v[jj + 1]),
                          c10, c11);
                     fma2(acc1[j + 2], acc1[j + 3], __uint_as_float(v[jj + 2]),
