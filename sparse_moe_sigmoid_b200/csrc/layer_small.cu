@@ -132,7 +132,6 @@ __device__ bool grid_sync(const SmallArgs& a, uint32_t& target, volatile uint32_
           ok = false;
           break;
         }
-        __nanosleep(32);
       }
     }
     *ok_s = ok ? 1u : 0u;
@@ -155,14 +154,16 @@ __device__ bool wait_ready(const SmallArgs& a, int g, uint32_t need, uint64_t li
       *abort_g = 1;
       return false;
     }
-    __nanosleep(32);
   }
 }
 
 // Router logits: CTAs split (8-token chunk) x (expert range); the chunk's x
-// rows sit in shared memory and each warp takes one expert at a time, lanes
-// striding K by 4 (float4 of the fp32 router row, exact BF16 x products, fp32
-// sums), then a warp reduction.
+// rows sit in shared memory. The six warps split K in six contiguous parts
+// and each lane strides its part by 4 (float4 of the fp32 router row, exact
+// BF16 products, fp32 sums), all of the CTA's experts at once so that their
+// row loads are in flight together; the six partial sums of each (expert,
+// token) are then added in warp order through shared memory.
+constexpr int kRouterMaxE = 8;  // experts per CTA per pass
 __device__ void phase_router(const SmallArgs& a, uint8_t* scratch) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nc = (a.T + kTokChunk - 1) / kTokChunk;
@@ -172,47 +173,65 @@ __device__ void phase_router(const SmallArgs& a, uint8_t* scratch) {
   const int t0 = chunk * kTokChunk, tn = min(kTokChunk, a.T - t0);
   const int e_lo = r * a.E / nb, e_hi = (r + 1) * a.E / nb;
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(scratch);
+  // partial sums [6 warps][kRouterMaxE][kTokChunk] after the x chunk
+  float* red = reinterpret_cast<float*>(scratch + (size_t)kTokChunk * a.d * 2);
   const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)t0 * a.d);
   uint4* dst = reinterpret_cast<uint4*>(xs);
   for (int i = threadIdx.x; i < tn * a.d / 8; i += kThreads) dst[i] = __ldg(src + i);
   __syncthreads();
-  constexpr int kPre = 8;  // float4 loads of the router row in flight per lane
-  for (int e = e_lo + warp; e < e_hi; e += kThreads / 32) {
-    const float* w = a.router + (size_t)e * a.d;
-    float acc[kTokChunk];
+  // this warp's K part: a multiple of 128 columns (a.d is a multiple of 256)
+  const int part = ((a.d / 128 + 5) / 6) * 128;
+  const int k_lo = warp * part, k_hi = min(a.d, k_lo + part);
+  for (int eb = e_lo; eb < e_hi; eb += kRouterMaxE) {
+    const int ne = min(kRouterMaxE, e_hi - eb);
+    float acc[kRouterMaxE][kTokChunk];
 #pragma unroll
-    for (int t = 0; t < kTokChunk; ++t) acc[t] = 0.f;
-    for (int c0 = lane * 4; c0 < a.d; c0 += 128 * kPre) {
-      float4 wv[kPre];
+    for (int q = 0; q < kRouterMaxE; ++q)
 #pragma unroll
-      for (int u = 0; u < kPre; ++u)
-        if (c0 + 128 * u < a.d) wv[u] = __ldg(reinterpret_cast<const float4*>(w + c0 + 128 * u));
+      for (int t = 0; t < kTokChunk; ++t) acc[q][t] = 0.f;
+    for (int c = k_lo + lane * 4; c < k_hi; c += 128) {
+      float4 wv[kRouterMaxE];
 #pragma unroll
-      for (int u = 0; u < kPre; ++u) {
-        const int c = c0 + 128 * u;
-        if (c < a.d) {
+      for (int q = 0; q < kRouterMaxE; ++q)
+        if (q < ne) wv[q] = __ldg(reinterpret_cast<const float4*>(a.router + (size_t)(eb + q) * a.d + c));
 #pragma unroll
-          for (int t = 0; t < kTokChunk; ++t) {
-            if (t < tn) {
-              const uint2 raw = *reinterpret_cast<const uint2*>(xs + (size_t)t * a.d + c);
-              const float2 p = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
-              const float2 q = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
-              acc[t] = fmaf(p.x, wv[u].x, acc[t]);
-              acc[t] = fmaf(p.y, wv[u].y, acc[t]);
-              acc[t] = fmaf(q.x, wv[u].z, acc[t]);
-              acc[t] = fmaf(q.y, wv[u].w, acc[t]);
+      for (int t = 0; t < kTokChunk; ++t) {
+        if (t < tn) {
+          const uint2 raw = *reinterpret_cast<const uint2*>(xs + (size_t)t * a.d + c);
+          const float2 p = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+          const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+#pragma unroll
+          for (int q = 0; q < kRouterMaxE; ++q) {
+            if (q < ne) {
+              acc[q][t] = fmaf(p.x, wv[q].x, acc[q][t]);
+              acc[q][t] = fmaf(p.y, wv[q].y, acc[q][t]);
+              acc[q][t] = fmaf(v.x, wv[q].z, acc[q][t]);
+              acc[q][t] = fmaf(v.y, wv[q].w, acc[q][t]);
             }
           }
         }
       }
     }
 #pragma unroll
-    for (int t = 0; t < kTokChunk; ++t) {
-      float v = acc[t];
+    for (int q = 0; q < kRouterMaxE; ++q) {
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-      if (lane == 0 && t < tn) a.logits[(size_t)(t0 + t) * a.E + e] = v;
+      for (int t = 0; t < kTokChunk; ++t) {
+        float v = acc[q][t];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == 0) red[(warp * kRouterMaxE + q) * kTokChunk + t] = v;
+      }
     }
+    __syncthreads();
+    if (threadIdx.x < ne * kTokChunk) {
+      const int q = threadIdx.x / kTokChunk, t = threadIdx.x % kTokChunk;
+      if (t < tn) {
+        float v = 0.f;
+        for (int w6 = 0; w6 < kThreads / 32; ++w6) v += red[(w6 * kRouterMaxE + q) * kTokChunk + t];
+        a.logits[(size_t)(t0 + t) * a.E + eb + q] = v;
+      }
+    }
+    __syncthreads();
   }
 }
 
@@ -485,6 +504,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t it = 0;
     bool run = true;
     for (int u = blockIdx.x; u < U && run; u += gridDim.x) {
+      // every gate/up unit precedes every down unit: from the first down
+      // unit on, lane 0 streams alone (box loads need no other lane, and a
+      // warp-wide loop with a shuffle and a warp barrier per stage measured
+      // slower for box loads)
+      if (u >= U1 && lane != 0) break;
       const SmallUnit su = decode_small(a, u, U1);
       int tok[4] = {};
       if (su.gu && 4 * lane < kBN) {
@@ -495,13 +519,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           tok[j] = a.row_token[su.un.row0 + (r < su.un.nvalid ? r : 0)];
         }
       }
-      if (!su.gu) {  // h rows of this group must all be stored first
-        if (lane == 0) {
-          run = wait_ready(a, su.un.g, ready_need(a, su.un.g), lim);
-          if (run) fence_proxy_async_global();
-        }
-        run = __shfl_sync(0xffffffffu, run, 0);
+      if (!su.gu) {  // lane 0 alone: h rows of this group must all be stored first
+        run = wait_ready(a, su.un.g, ready_need(a, su.un.g), lim);
         if (!run) break;
+        fence_proxy_async_global();
+        for (int kb = 0; kb < su.kb; ++kb, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim)) {
+            run = false;
+            break;
+          }
+          uint8_t* st = smem + s * kStage;
+          mbar_arrive_expect_tx(&full[s], kStage);
+          tma_load_3d(st, &tmD, &full[s], kb * kK, su.un.mt * 256, su.un.g);
+          tma_load_3d(st + kA, &tmD, &full[s], kb * kK, su.un.mt * 256 + 128, su.un.g);
+          tma_load_2d(st + 2 * kA, &tmH, &full[s], kb * kK, su.un.row0);
+          *issued = it + 1;
+        }
+        continue;
       }
       for (int kb = 0; kb < su.kb; ++kb, ++it) {
         const int s = it % kStages;
@@ -512,16 +548,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* st = smem + s * kStage;
         if (lane == 0) {
           mbar_arrive_expect_tx(&full[s], kStage);
-          if (su.gu) {
-            tma_load_3d(st, &tmG, &full[s], kb * kK, su.un.mt * 128, su.un.g);
-            tma_load_3d(st + kA, &tmU, &full[s], kb * kK, su.un.mt * 128, su.un.g);
-          } else {
-            tma_load_3d(st, &tmD, &full[s], kb * kK, su.un.mt * 256, su.un.g);
-            tma_load_3d(st + kA, &tmD, &full[s], kb * kK, su.un.mt * 256 + 128, su.un.g);
-            tma_load_2d(st + 2 * kA, &tmH, &full[s], kb * kK, su.un.row0);
-          }
+          tma_load_3d(st, &tmG, &full[s], kb * kK, su.un.mt * 128, su.un.g);
+          tma_load_3d(st + kA, &tmU, &full[s], kb * kK, su.un.mt * 128, su.un.g);
         }
-        if (su.gu && 4 * lane < kBN)
+        if (4 * lane < kBN)
           tma_gather4(st + 2 * kA + 4 * lane * 128, &tmX, &full[s], kb * kK, tok[0], tok[1],
                       tok[2], tok[3]);
         __syncwarp();
@@ -804,7 +834,9 @@ bool small_layer_supported(const Dims& dm, int64_t T, int64_t max_t) {
   const int kb2 = dm.fp8 ? dm.f / 128 : dm.f / 64;
   if (kb1 > kMaxKB || kb2 > kMaxKB) return false;
   // the router's x chunk must fit the shared-memory ring
-  if (static_cast<size_t>(kTokChunk) * dm.d * 2 > static_cast<size_t>(kStages) * kStage) return false;
+  if (static_cast<size_t>(kTokChunk) * dm.d * 2 + 6 * kRouterMaxE * kTokChunk * 4 >
+      static_cast<size_t>(kStages) * kStage)
+    return false;
   return true;
 }
 
