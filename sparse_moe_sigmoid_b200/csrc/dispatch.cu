@@ -32,10 +32,13 @@
 
 namespace smoe {
 
-static int pick_bn(double want, const int* cands, int n) {
-  for (int i = 0; i < n; ++i)
+static int pick_bn(double want, const int* cands, int n, int cap = 1 << 30) {
+  int last = cands[0];
+  for (int i = 0; i < n && cands[i] <= cap; ++i) {
+    last = cands[i];
     if (cands[i] >= want) return cands[i];
-  return cands[n - 1];
+  }
+  return last;
 }
 
 // Row-tile height: the smallest supported height >= SMOE_BN_FACTOR x the mean
@@ -54,6 +57,17 @@ static int pick_bn(double want, const int* cands, int n) {
 #ifndef SMOE_FP8_GATHER_MAX_BN
 #define SMOE_FP8_GATHER_MAX_BN 32
 #endif
+// tallest FP8 row tiles (tuning constants): gate/up 96 (three promotion
+// warpgroups, two TMEM partial buffers), down 192. Measured against shorter
+// caps at T = 16384 (same box): gate/up capped at 64 rows with four
+// promotion warpgroups (four partial buffers) 12.30 vs 11.38 ms; down capped
+// at 128 rows (four partial buffers) 7.50 vs 6.32 ms; T = 4096 likewise.
+#ifndef SMOE_FP8_GU_MAX_BN
+#define SMOE_FP8_GU_MAX_BN 96
+#endif
+#ifndef SMOE_FP8_DOWN_MAX_BN
+#define SMOE_FP8_DOWN_MAX_BN 192
+#endif
 // mean rows per routed expert (T k / E); every token's row in each shared
 // group when there are no routed experts
 static double rows_per_group(const Dims& dm, int64_t T) {
@@ -65,7 +79,7 @@ GemmPlan plan_gate_up(const Dims& dm, int64_t T) {
   static const int fp8_bn[] = {16, 32, 64, 96};
   const double want = SMOE_BN_FACTOR * rows_per_group(dm, T);
   GemmPlan p;
-  p.bn = dm.fp8 ? pick_bn(want, fp8_bn, 4) : pick_bn(want, bf16_bn, 9);
+  p.bn = dm.fp8 ? pick_bn(want, fp8_bn, 4, SMOE_FP8_GU_MAX_BN) : pick_bn(want, bf16_bn, 9);
   p.na = 2;
   p.pair = !dm.fp8 && pair_bn_supported(p.bn) && dm.f % 256 == 0;
   p.gather = !p.pair && p.bn <= (dm.fp8 ? SMOE_FP8_GATHER_MAX_BN : kGatherMaxBn);
@@ -84,7 +98,7 @@ GemmPlan plan_down(const Dims& dm, int64_t T) {
   static const int fp8_bn[] = {16, 32, 64, 128, 192};
   const double want = SMOE_BN_FACTOR * rows_per_group(dm, T);
   GemmPlan p;
-  p.bn = dm.fp8 ? pick_bn(want, fp8_bn, 5) : pick_bn(want, bf16_bn, 9);
+  p.bn = dm.fp8 ? pick_bn(want, fp8_bn, 5, SMOE_FP8_DOWN_MAX_BN) : pick_bn(want, bf16_bn, 9);
   p.pair = !dm.fp8 && pair_bn_supported(p.bn) && dm.d % 256 == 0 && dm.f % 128 == 0;
   p.gather = false;  // h rows are written in expert order by gate/up
   // two weight tiles per unit: FP8 up to 64 rows (measured: T=128 down GEMM

@@ -50,6 +50,12 @@ namespace smoe {
 
 using namespace sm100;
 
+// promotion warpgroups of the 64-row FP8 gate/up tile (a tuning constant:
+// two hold 32 columns a thread, four hold 16 with fewer registers each;
+// four measured no faster where 64-row tiles run)
+#ifndef SMOE_FP8_GU64_NPG
+#define SMOE_FP8_GU64_NPG 2
+#endif
 constexpr int kFp8MaxKBlocks = 64;  // hidden_size and moe_intermediate_size <= 8192
 constexpr int kPromMaxStages = 12;
 constexpr int kPromSmemBudget = 227 * 1024 - 2048;
@@ -98,8 +104,16 @@ struct PromCfg {
   static constexpr int scale_bytes(int kb) {
     return !FP8 ? 0 : kPreMul ? (kTwoA ? 2 : 1) * kb * BN * 4 : (kb * BN + 2 * kb) * 4;
   }
+  // Tall FP8 tiles (three promotion warpgroups) leave 44 KB of the SM's
+  // shared memory to L1, one ring stage fewer: the per-tile scale staging and
+  // the unit decoding read through it. Measured at T = 16384 in two runs:
+  // gate/up (96-row tiles, 4 -> 3 stages) 11.6-11.8 -> 11.1-11.2 ms, down
+  // (192-row tiles, 5 -> 4 stages) 6.5-6.6 -> 6.3 ms; T = 4096 3.90 -> 3.76 ms
+  // (gate/up); unchanged at T = 1024.
+  static constexpr int kL1Reserve = FP8 && NPG >= 3 ? 45056 : 0;
   static constexpr int stages(int kb) {
-    const int n = (kPromSmemBudget - kBarrierBytes - scale_bytes(kb) - kAmaxBytes) / kStage;
+    const int n =
+        (kPromSmemBudget - kL1Reserve - kBarrierBytes - scale_bytes(kb) - kAmaxBytes) / kStage;
     return n > kPromMaxStages ? kPromMaxStages : n;
   }
   static constexpr int smem(int kb) {
@@ -612,7 +626,7 @@ cudaError_t launch_gemm_fp8(moe_handle* h, bool gated, const GemmPlan& p, cudaSt
     switch (p.bn) {
       case 16: return launch_one<16, true, true, 1>(h, g, u, b, a, s);
       case 32: return launch_one<32, true, true, 1>(h, g, u, b, a, s);
-      case 64: return launch_one<64, true, true, 2>(h, g, u, b, a, s);
+      case 64: return launch_one<64, true, true, SMOE_FP8_GU64_NPG>(h, g, u, b, a, s);
       case 96: return launch_one<96, true, true, 3>(h, g, u, b, a, s);
       default: return cudaErrorInvalidValue;
     }
