@@ -471,11 +471,14 @@ def run_native(args, wl):
     torch.cuda.empty_cache()
 
     y = torch.empty_like(x)
-    m = measure(smoe, h, x, y, T, fmt, shape, args, dev, args.config)
+    # DRAM traffic figures belong to the full-size workloads they were taken on
+    traffic_key = None if wl.get("reduced") else args.config
+    m = measure(smoe, h, x, y, T, fmt, shape, args, dev, traffic_key)
     pre = None
     if T_pre:
         xp = x_all[:T_pre].contiguous()
-        pre = measure(smoe, h, xp, torch.empty_like(xp), T_pre, fmt, shape, args, dev, "prefill")
+        pre = measure(smoe, h, xp, torch.empty_like(xp), T_pre, fmt, shape, args, dev,
+                      None if wl.get("reduced") else "prefill")
         pre = {"workload": f"K2 MoE layer prefill, T={T_pre} tokens, {fmt.upper()} experts "
                            "(same weights and handle)",
                "ms_per_step": pre["ms_per_step"], "value": pre["value"], "unit": UNIT,
@@ -573,6 +576,7 @@ def main(argv=None):
         E = args.experts or synth.K2.n_routed_experts
         wl["shape"] = synth.LayerShape(n_routed_experts=E)
         wl["desc"] += f" [reduced case: T={wl['T']}, {E} routed experts]"
+        wl["reduced"] = True
     if args.steps is None:
         args.steps = (400 if wl["T"] <= 1024 else 100) if args.impl == "native" else 5
     if args.warmup < 3 and args.impl == "native":

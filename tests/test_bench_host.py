@@ -117,3 +117,20 @@ def test_reference_arm_prints_the_contract_line(capsys):
     assert e2e["value"] == j["value"] and e2e["unit"] == j["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
     assert j["config"]["tokens"] == 8 and j["config"]["n_routed_experts"] == 16
+
+
+def test_traffic_only_for_the_workload_it_was_taken_on(tmp_path, monkeypatch):
+    # a committed traffic figure counts only for its own full-size workload and
+    # only while the GEMM sources it was measured on are unchanged
+    src = bench.kernel_src_hash("gemm_gate_up")
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "traffic.json").write_text(
+        '{"decode": {"gemm_gate_up": {"bytes_per_launch": 123, "src": "%s"}},'
+        ' "prefill": {"gemm_gate_up": {"bytes_per_launch": 456, "src": "stale"}}}' % src)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_src_hash", lambda k: src)
+    assert bench.traffic_for("gemm_gate_up", "decode") == 123
+    assert bench.traffic_for("gemm_gate_up", "prefill") is None  # sources changed since
+    assert bench.traffic_for("gemm_gate_up", None) is None  # a reduced case
+    assert bench.traffic_for("gemm_down", "decode") is None
