@@ -118,14 +118,21 @@ def barrier(device):
 
 
 # ------------------------------------------------------------------- clocks
+def smi_device(local: int) -> str:
+    """The nvidia-smi id (-i) of CUDA device `local`: CUDA_VISIBLE_DEVICES
+    renumbers devices, nvidia-smi does not (it takes the listed index or UUID)."""
+    vis = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    return vis[local] if local < len(vis) else str(local)
+
+
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons while running."""
     Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, gpu: str):
+        self.gpu = gpu
         self.proc = None
         self.lines = []
 
@@ -308,7 +315,7 @@ def measure(smoe, h, x, y, T, fmt, shape, args, dev, config_name):
     # the timed steps: plain forwards, as a caller runs them (the library
     # replays them as a CUDA graph from the second call on)
     n0 = smoe.moe_launch_count(h)
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(smi_device(local))
     clocks.start()
     time.sleep(0.3)
     barrier(dev)

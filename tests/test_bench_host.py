@@ -134,3 +134,12 @@ def test_traffic_only_for_the_workload_it_was_taken_on(tmp_path, monkeypatch):
     assert bench.traffic_for("gemm_gate_up", "prefill") is None  # sources changed since
     assert bench.traffic_for("gemm_gate_up", None) is None  # a reduced case
     assert bench.traffic_for("gemm_down", "decode") is None
+
+
+def test_clock_sampler_follows_cuda_visible_devices(monkeypatch):
+    monkeypatch.delenv("CUDA_VISIBLE_DEVICES", raising=False)
+    assert bench.smi_device(1) == "1"
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "5,3")
+    assert bench.smi_device(0) == "5" and bench.smi_device(1) == "3"
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "GPU-aaaa")
+    assert bench.smi_device(0) == "GPU-aaaa"
