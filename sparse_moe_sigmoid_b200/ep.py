@@ -110,10 +110,21 @@ class LibraryEP:
     the router (moe_router_topk_noalloc, over all experts), this rank's slice
     of the routed experts (a handle with k = 1, weight 1 and the expert forced
     per row, so each row's output is E_e(x)), the shared expert (a handle with
-    no routed experts) and the combine (moe_combine_rows)."""
+    no routed experts) and the combine (moe_combine_rows). FP8 weights take
+    their block scales (the routed ones sliced like the weights). Group-limited
+    routing (n_group > 1) is refused: the allocation-free router routes over
+    all experts with n_group = 1."""
 
     def __init__(self, smoe, cfg, router_weight, bias, gate, up, down, shared_gate=None,
-                 shared_up=None, shared_down=None, max_tokens=8192, group=None, device=None):
+                 shared_up=None, shared_down=None, max_tokens=8192, group=None, device=None,
+                 gate_scale=None, up_scale=None, down_scale=None, shared_gate_scale=None,
+                 shared_up_scale=None, shared_down_scale=None):
+        if cfg.n_group > 1:
+            raise ValueError("expert parallelism here routes with n_group = 1; "
+                             f"the config asks for n_group = {cfg.n_group}")
+        fp8 = cfg.weight_format == smoe.MOE_WEIGHT_FP8_E4M3_BLOCK
+        if fp8 and (gate_scale is None or up_scale is None or down_scale is None):
+            raise ValueError("FP8 expert weights need their block scales")
         self.smoe, self.group = smoe, group
         world = dist.get_world_size(group)
         rank = dist.get_rank(group)
@@ -123,26 +134,33 @@ class LibraryEP:
         lo = rank * per
         self.router_weight, self.bias = router_weight, bias
         dev = router_weight.device if device is None else device
+        dev_index = dev.index if dev.index is not None else torch.cuda.current_device()
         d = cfg.hidden_size
+        fmt = dict(weight_format=cfg.weight_format,
+                   weight_block_size=tuple(cfg.weight_block_size))
+        sl = (lambda t: None if t is None else t[lo:lo + per])
         ex_cfg = smoe.moe_config_init_k2(
             hidden_size=d, moe_intermediate_size=cfg.moe_intermediate_size,
             n_routed_experts=per, num_experts_per_tok=1, n_shared_experts=0,
             norm_topk_prob=1, routed_scaling_factor=1.0,
-            max_tokens=max(1, world * max_tokens * self.k))
-        self.ex = smoe.moe_create(ex_cfg, dev.index or 0)
+            max_tokens=max(1, world * max_tokens * self.k), **fmt)
+        self.ex = smoe.moe_create(ex_cfg, dev_index)
         zero_w = torch.zeros((per, d), dtype=torch.float32, device=dev)  # routing is forced
         zero_b = torch.zeros((per,), dtype=torch.float32, device=dev)
-        smoe.moe_load_weights(self.ex, zero_w, zero_b, gate[lo:lo + per], up[lo:lo + per],
-                              down[lo:lo + per])
+        smoe.moe_load_weights(self.ex, zero_w, zero_b, sl(gate), sl(up), sl(down),
+                              gate_scale=sl(gate_scale), up_scale=sl(up_scale),
+                              down_scale=sl(down_scale))
         self.sh = None
         if shared_gate is not None and cfg.n_shared_experts > 0:
             sh_cfg = smoe.moe_config_init_k2(
                 hidden_size=d, moe_intermediate_size=cfg.moe_intermediate_size,
                 n_routed_experts=0, num_experts_per_tok=0,
-                n_shared_experts=cfg.n_shared_experts, max_tokens=max(1, max_tokens))
-            self.sh = smoe.moe_create(sh_cfg, dev.index or 0)
+                n_shared_experts=cfg.n_shared_experts, max_tokens=max(1, max_tokens), **fmt)
+            self.sh = smoe.moe_create(sh_cfg, dev_index)
             smoe.moe_load_weights(self.sh, None, None, None, None, None, shared_gate, shared_up,
-                                  shared_down)
+                                  shared_down, shared_gate_scale=shared_gate_scale,
+                                  shared_up_scale=shared_up_scale,
+                                  shared_down_scale=shared_down_scale)
         torch.cuda.synchronize(dev)
 
     def route(self, x):

@@ -128,3 +128,15 @@ def test_plan_rejects_uneven_slices_and_bad_ids():
         ep.make_plan(torch.zeros((2, 2), dtype=torch.int64), 10, 4)
     with pytest.raises(ValueError):
         ep.make_plan(torch.tensor([[0, 16]]), 16, 2)
+
+
+def test_library_ep_refuses_what_its_router_cannot_do():
+    # the checks run before any device work, so no GPU is needed
+    import sparse_moe_sigmoid_b200 as smoe
+    from sparse_moe_sigmoid_b200 import ep
+    cfg = smoe.moe_config_init_k2(n_group=8, topk_group=4)
+    with pytest.raises(ValueError, match="n_group"):
+        ep.LibraryEP(smoe, cfg, None, None, None, None, None)
+    cfg = smoe.moe_config_init_k2(weight_format=smoe.MOE_WEIGHT_FP8_E4M3_BLOCK)
+    with pytest.raises(ValueError, match="block scales"):
+        ep.LibraryEP(smoe, cfg, None, None, None, None, None)

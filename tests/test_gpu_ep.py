@@ -59,17 +59,21 @@ def test_combine_rows_matches_the_oracle(smoe):
     assert np.max(np.abs(gu.f64(y0) - want0)) / np.max(np.abs(want0)) <= 2 ** -8
 
 
-@pytest.mark.parametrize("fmt", ["bf16"])
+@pytest.mark.parametrize("fmt", ["bf16", "fp8"])
 @pytest.mark.parametrize("T", [1, 40, 300])
 def test_ep_rank_on_one_gpu_matches_the_oracle(smoe, nccl_world1, fmt, T):
     from sparse_moe_sigmoid_b200 import ep
     layer = gu.make_layer(synth.TINY, 300, fmt)
-    cfg = smoe.moe_config_init_k2(hidden_size=256, moe_intermediate_size=128,
-                                  n_routed_experts=16, num_experts_per_tok=4,
-                                  n_shared_experts=1)
+    cfg = smoe.moe_config_init_k2(
+        hidden_size=256, moe_intermediate_size=128, n_routed_experts=16, num_experts_per_tok=4,
+        n_shared_experts=1,
+        weight_format=smoe.MOE_WEIGHT_BF16 if fmt == "bf16" else smoe.MOE_WEIGHT_FP8_E4M3_BLOCK)
     ew = layer.ew
     L = ep.LibraryEP(smoe, cfg, layer.Wg, layer.b, ew.gate, ew.up, ew.down, ew.shared_gate,
-                     ew.shared_up, ew.shared_down, max_tokens=300)
+                     ew.shared_up, ew.shared_down, max_tokens=300,
+                     gate_scale=ew.gate_scale, up_scale=ew.up_scale, down_scale=ew.down_scale,
+                     shared_gate_scale=ew.shared_gate_scale, shared_up_scale=ew.shared_up_scale,
+                     shared_down_scale=ew.shared_down_scale)
     try:
         x = layer.x[:T].contiguous()
         ids, w = L.route(x)
