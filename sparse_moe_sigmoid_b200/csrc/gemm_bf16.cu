@@ -363,10 +363,18 @@ cudaError_t launch_gemm_bf16(moe_handle* h, bool gated, const GemmPlan& p, cudaS
   const CUtensorMap& b = h->tm_h[bi];
   const CUtensorMap& w = h->tm_down;
   if (p.na == 1) {
+    // one 128-row weight tile per unit: short tiles, and every tile height
+    // when hidden_size is an odd multiple of 128 (no 256-feature units)
     switch (p.bn) {
       case 16: return launch_one<16, 1, false>(h, w, w, b, a, s);
       case 32: return launch_one<32, 1, false>(h, w, w, b, a, s);
       case 64: return launch_one<64, 1, false>(h, w, w, b, a, s);
+      case 96: return launch_one<96, 1, false>(h, w, w, b, a, s);
+      case 128: return launch_one<128, 1, false>(h, w, w, b, a, s);
+      case 160: return launch_one<160, 1, false>(h, w, w, b, a, s);
+      case 192: return launch_one<192, 1, false>(h, w, w, b, a, s);
+      case 224: return launch_one<224, 1, false>(h, w, w, b, a, s);
+      case 256: return launch_one<256, 1, false>(h, w, w, b, a, s);
       default: return cudaErrorInvalidValue;
     }
   }

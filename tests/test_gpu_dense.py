@@ -76,3 +76,12 @@ def test_k2_dense_ffn(smoe, fmt, T):
     err, _ = _run_dense(smoe, _dense_shape(7168, 2048, 9), fmt, T, toks)
     print(f"dense {fmt} T={T}: {len(toks)} tokens, max rel err {err:.2e}")
     assert err <= gu.TOL[fmt], err
+
+
+@pytest.mark.parametrize("fmt", ["bf16", "fp8"])
+def test_dense_ffn_odd_sizes(smoe, fmt):
+    """d = 384 and intermediate 2 x 384 (odd multiples of 128: no 256-feature
+    down tiles, no CTA pairs): every token."""
+    err, launches = _run_dense(smoe, _dense_shape(384, 384, 2), fmt, 100)
+    assert err <= gu.TOL[fmt], err
+    assert launches == 5
