@@ -7,7 +7,8 @@ chosen to reach a path the K2 shapes do not: sizes that are odd multiples of
 128 (no 256-feature down tiles, no CTA pairs), a single or very few experts
 (tall row tiles, FP8 promotion with three warpgroups), many experts, k = 1,
 odd and maximal k, the longest FP8 K (64 blocks), group-limited routing in
-FP8, and the single launch (the dense layer's odd sizes are in
+FP8, unnormalised weights and other scaling factors, 16 shared groups, and
+the single launch (the dense layer's odd sizes are in
 test_gpu_dense.py). Every token's output is compared
 (T <= 1000), with the acceptance rule of the other parity tests, and the
 dispatch's row order is checked against the routing.
@@ -38,6 +39,16 @@ CASES = [
     ("f8192_fp8", S(128, 8192, 4, 2, 1), 20, "fp8", 0),
     ("single_launch_bf16", S(512, 256, 24, 4, 1), 16, "bf16", 128),
     ("single_launch_fp8", S(512, 256, 24, 4, 1), 16, "fp8", 128),
+    # routing settings other than K2's: weights not normalised, other scales
+    ("no_norm_scale1", S(512, 256, 32, 6, 1, routed_scaling_factor=1.0, norm_topk_prob=False),
+     200, "bf16", 0),
+    ("no_norm_scale2p5_fp8", S(512, 256, 32, 6, 0, routed_scaling_factor=2.5,
+                               norm_topk_prob=False), 200, "fp8", 0),
+    ("grouped_top1", S(256, 128, 16, 1, 1, n_group=4, topk_group=1), 100, "bf16", 0),
+    ("sixteen_shared", S(256, 128, 8, 2, 16), 50, "bf16", 0),
+    ("single_launch_no_norm", S(512, 256, 24, 4, 1, norm_topk_prob=False), 16, "bf16", 128),
+    ("single_launch_grouped_fp8", S(512, 256, 24, 4, 1, n_group=4, topk_group=2), 16, "fp8",
+     128),
 ]
 
 
