@@ -241,10 +241,11 @@ __global__ void __launch_bounds__(256) dispatch_fp8_kernel(
 // row (blocks [0, place_blocks)) writes the pair's row (pair_row) and the
 // row's token (row_token), which the gate/up GEMMs use to gather x rows; no
 // row is copied. FP8: the blocks after those quantise each token's x row
-// once (one warp per token) into rows [0, T) of xq / xs, which the GEMMs
+// once (qparts warps per token) into rows [0, T) of xq / xs, which the GEMMs
 // gather from instead of x.
 __global__ void __launch_bounds__(256) dispatch_kernel(
     const __nv_bfloat16* __restrict__ x, int T, int d, int k, int E, int items, int place_blocks,
+    int qparts,
     const int32_t* __restrict__ ids, const uint32_t* __restrict__ bitmap,
     const int32_t* __restrict__ word_prefix, const int32_t* __restrict__ offsets, int W,
     int32_t* __restrict__ pair_row, int32_t* __restrict__ row_token, uint8_t* __restrict__ xq,
@@ -259,27 +260,42 @@ __global__ void __launch_bounds__(256) dispatch_kernel(
     return;
   }
   const int lane = threadIdx.x & 31;
-  const int t = ((blockIdx.x - place_blocks) * blockDim.x + threadIdx.x) >> 5;
+  const int qw = ((blockIdx.x - place_blocks) * blockDim.x + threadIdx.x) >> 5;
+  const int t = qw / qparts;
   if (t >= T) return;
-  quant_row_e4m3(x + (size_t)t * d, d, xq + (size_t)t * d, xs + (size_t)t * (d / 128), lane);
+  quant_row_e4m3(x + (size_t)t * d, d, xq + (size_t)t * d, xs + (size_t)t * (d / 128), lane,
+                 qw - t * qparts, qparts);
 }
 
 // Dynamic activation quantisation of a dense [rows, d] BF16 matrix.
 __global__ void __launch_bounds__(256) act_quant_kernel(const __nv_bfloat16* __restrict__ x,
-                                                        int64_t rows, int d,
+                                                        int64_t rows, int d, int parts,
                                                         uint8_t* __restrict__ q,
                                                         float* __restrict__ s) {
   const int lane = threadIdx.x & 31;
-  const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t r = w / parts;
   if (r >= rows) return;
-  quant_row_e4m3(x + r * d, d, q + r * d, s + r * (d / 128), lane);
+  quant_row_e4m3(x + r * d, d, q + r * d, s + r * (d / 128), lane, static_cast<int>(w - r * parts),
+                 parts);
+}
+
+// Warps per row of the e4m3 quantisation: one per row when there are rows
+// enough to fill the GPU (~16 warps per SM), else up to one per pair of
+// 128-column groups.
+static int quant_parts(int64_t rows, int d, int sms = 148) {
+  const int64_t want = 16 * static_cast<int64_t>(sms);
+  const int64_t most = (d / 128 + 1) / 2;
+  const int64_t p = rows > 0 ? want / rows : most;
+  return static_cast<int>(p < 1 ? 1 : (p > most ? most : p));
 }
 
 cudaError_t launch_act_quant(const void* x, int64_t rows, int d, uint8_t* q, float* s,
                              cudaStream_t st) {
-  const int64_t blocks = (rows * 32 + 255) / 256;
+  const int parts = quant_parts(rows, d);
+  const int64_t blocks = (rows * parts * 32 + 255) / 256;
   act_quant_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(x), rows, d, q, s);
+      static_cast<const __nv_bfloat16*>(x), rows, d, parts, q, s);
   return cudaGetLastError();
 }
 
@@ -290,9 +306,11 @@ cudaError_t launch_dispatch(moe_handle* h, const void* x, int T, bool gather, cu
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   if (gather) {
     const int place_blocks = (items + 255) / 256;
-    const int quant_blocks = dm.fp8 ? (T * 32 + 255) / 256 : 0;
+    const int qparts = dm.fp8 ? quant_parts(T, dm.d, h->num_sms) : 1;
+    const int quant_blocks =
+        dm.fp8 ? static_cast<int>(((int64_t)T * qparts * 32 + 255) / 256) : 0;
     dispatch_kernel<<<place_blocks + quant_blocks, 256, 0, s>>>(
-        xb, T, dm.d, dm.k, dm.E, items, place_blocks, h->ws.ids, h->ws.bitmap,
+        xb, T, dm.d, dm.k, dm.E, items, place_blocks, qparts, h->ws.ids, h->ws.bitmap,
         h->ws.word_prefix, h->ws.offsets, W, h->ws.pair_row, h->ws.row_token,
         static_cast<uint8_t*>(h->ws.xp), h->ws.xs);
   } else {

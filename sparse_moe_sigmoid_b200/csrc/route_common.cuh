@@ -253,13 +253,17 @@ __device__ __forceinline__ int place_row(int i, int T, int k, int E, const int32
   return offsets[E + s] + t;
 }
 
-// One row of d BF16 values -> d e4m3 codes + d/128 fp32 scales, by one warp:
-// each half-warp takes one 128-column group (16 lanes x 8 values).
+// One row of d BF16 values -> d e4m3 codes + d/128 fp32 scales: each
+// half-warp takes one 128-column group (16 lanes x 8 values). A row may be
+// shared by `parts` warps, warp `part` taking the group pairs part,
+// part + parts, ... (few rows: the groups' loads then run in parallel
+// instead of one after another in a single warp).
 __device__ __forceinline__ void quant_row_e4m3(const __nv_bfloat16* __restrict__ src, int d,
                                                uint8_t* __restrict__ dst,
-                                               float* __restrict__ scales, int lane) {
+                                               float* __restrict__ scales, int lane,
+                                               int part = 0, int parts = 1) {
   const int ngroups = d / 128;
-  for (int g0 = 0; g0 < ngroups; g0 += 2) {
+  for (int g0 = 2 * part; g0 < ngroups; g0 += 2 * parts) {
     const int gi = g0 + (lane >> 4);
     const bool active = gi < ngroups;
     const int col = gi * 128 + (lane & 15) * 8;
