@@ -21,9 +21,9 @@
 //
 // Measured against the phase kernels on one B200: the routing phases are
 // cheaper here, but the gate/up tiles stream 10-25% slower (decode T = 64:
-// 3.62 vs 3.38 ms; FP8 T = 16: 1.02 vs 0.87 ms); only FP8 T = 1 comes out
-// ahead (0.127 vs 0.129 ms). It is therefore opt-in per handle
-// (single_launch_max_tokens, default 0).
+// 3.62 vs 3.38 ms; FP8 T = 16: 1.02 vs 0.87 ms; FP8 T = 1: 0.127 vs
+// 0.118 ms). It is therefore opt-in per handle (single_launch_max_tokens,
+// default 0).
 //
 // Launch: cooperative (every CTA resident at once, or the launch fails), one
 // CTA of six warps per SM: warp 0 loads (TMA), warp 1 owns TMEM and issues
