@@ -138,6 +138,191 @@ __global__ void __launch_bounds__(256) router_topk_kernel(TopkArgs a) {
   route_token(a, t, group_rows[threadIdx.x >> 5], lane);
 }
 
+// Few tokens: one warp's k rounds over all E experts are a long serial chain
+// (~2800 instructions for K2's E = 384, k = 8, one token measured at ~14 us).
+// Here four warps share a token (a 128-thread group, two tokens per CTA):
+// warp w takes the contiguous experts [w * chunk, (w + 1) * chunk), chunk =
+// ceil(E / 4) <= 128, four per lane; it adds their partial logits in slice
+// order and forms scores and keys exactly as route_token, then extracts its
+// own k best (key descending, the lower expert first on equal keys) into
+// shared memory; warp 0 of the group extracts the k best of those 4k
+// candidates the same way and finishes as route_token does. The k best of all
+// experts are among the candidates and the order is total, so the experts,
+// their order, the weights and the bookkeeping are route_token's bit for bit.
+// A token with a NaN key goes to route_token (its fallback for keys that
+// compare false needs every expert). Unforced routing with n_group = 1 only.
+constexpr int kSmallTopkWarps = 4;
+constexpr int kSmallTopkPerLane = kMaxExperts / 32 / kSmallTopkWarps;
+constexpr int kSmallTopkMaxT = 256;
+
+__global__ void __launch_bounds__(256) router_topk_small_kernel(TopkArgs a) {
+  constexpr int kC = kSmallTopkWarps * kMaxTopK;  // candidates per token, at most
+  __shared__ float c_key[2][kC], c_sc[2][kC];
+  __shared__ int c_id[2][kC];
+  __shared__ int c_nan[2];
+  const unsigned full = 0xffffffffu;
+  const int g = threadIdx.x >> 7;        // token slot of this CTA
+  const int w = (threadIdx.x >> 5) & 3;  // warp within the token's group
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 2 + g;
+  const bool live = t < a.T;
+  const int E = a.E, k = a.k;
+  const int chunk = (E + kSmallTopkWarps - 1) / kSmallTopkWarps;
+  const int e0 = w * chunk;
+  const int e1 = E < e0 + chunk ? E : e0 + chunk;
+  if (threadIdx.x < 2) c_nan[threadIdx.x] = 0;
+  __syncthreads();
+
+  float key[kSmallTopkPerLane], sc[kSmallTopkPerLane];
+  bool nan = false;
+#pragma unroll
+  for (int i = 0; i < kSmallTopkPerLane; ++i) {
+    key[i] = -INFINITY;
+    sc[i] = 0.f;
+  }
+  if (live) {
+    float lg[kSmallTopkPerLane];
+#pragma unroll
+    for (int i = 0; i < kSmallTopkPerLane; ++i) lg[i] = 0.f;
+#pragma unroll 4
+    for (int s = 0; s < a.splits; ++s) {
+      const float* ps = a.part + ((size_t)s * a.T + t) * E;
+      float v[kSmallTopkPerLane];
+#pragma unroll
+      for (int i = 0; i < kSmallTopkPerLane; ++i) {
+        const int e = e0 + lane + 32 * i;
+        v[i] = e < e1 ? ps[e] : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < kSmallTopkPerLane; ++i) lg[i] += v[i];
+    }
+#pragma unroll
+    for (int i = 0; i < kSmallTopkPerLane; ++i) {
+      const int e = e0 + lane + 32 * i;
+      if (e < e1) {
+        const float l = lg[i];
+        if (a.logits_out) a.logits_out[(size_t)t * E + e] = l;
+        const float p = 1.f / (1.f + expf(-l));
+        sc[i] = p;
+        key[i] = p + a.bias[e];
+        nan |= key[i] != key[i];
+      }
+    }
+  }
+  if (__any_sync(full, nan) && lane == 0) c_nan[g] = 1;
+
+  // this warp's k best: round j's winner is kept by lane j
+  float my_key = -INFINITY, my_sc = 0.f;
+  int my_id = 0x7fffffff;
+  uint32_t taken = 0;
+  for (int j = 0; j < k; ++j) {
+    float bk = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < kSmallTopkPerLane; ++i) {
+      const int e = e0 + lane + 32 * i;
+      if (e < e1 && !((taken >> i) & 1u) && (key[i] > bk || (key[i] == bk && e < bi))) {
+        bk = key[i];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ok = __shfl_xor_sync(full, bk, off);
+      const int oi = __shfl_xor_sync(full, bi, off);
+      if (ok > bk || (ok == bk && oi < bi)) {
+        bk = ok;
+        bi = oi;
+      }
+    }
+    float v = 0.f;
+    if (bi < e1) {  // a winner (else no expert of this warp is left)
+      const int r = bi - e0;
+      if ((r & 31) == lane) taken |= 1u << (r >> 5);
+#pragma unroll
+      for (int i = 0; i < kSmallTopkPerLane; ++i)
+        if (i == (r >> 5)) v = sc[i];
+      v = __shfl_sync(full, v, r & 31);
+    }
+    if (lane == j) {
+      my_key = bk;
+      my_id = bi;
+      my_sc = v;
+    }
+  }
+  if (lane < k) {
+    c_key[g][w * k + lane] = my_key;
+    c_sc[g][w * k + lane] = my_sc;
+    c_id[g][w * k + lane] = my_id;
+  }
+  __syncthreads();
+  if (w != 0 || !live) return;
+  if (c_nan[g]) {  // NaN keys: the one-warp routine and its fallback
+    route_token(a, t, &c_key[g][0], lane);
+    return;
+  }
+
+  // the k best of the 4k candidates (candidate c on lane c % 32, slot c / 32)
+  const int nc = kSmallTopkWarps * k;
+  float ck[kSmallTopkWarps], cs[kSmallTopkWarps];
+  int ci[kSmallTopkWarps];
+#pragma unroll
+  for (int i = 0; i < kSmallTopkWarps; ++i) {
+    const int c = lane + 32 * i;
+    ck[i] = c < nc ? c_key[g][c] : -INFINITY;
+    cs[i] = c < nc ? c_sc[g][c] : 0.f;
+    ci[i] = c < nc ? c_id[g][c] : 0x7fffffff;
+  }
+  my_sc = 0.f;
+  my_id = 0;
+  taken = 0;
+  for (int j = 0; j < k; ++j) {
+    float bk = -INFINITY;
+    int bi = 0x7fffffff, bc = 0;
+#pragma unroll
+    for (int i = 0; i < kSmallTopkWarps; ++i) {
+      if (!((taken >> i) & 1u) && (ck[i] > bk || (ck[i] == bk && ci[i] < bi))) {
+        bk = ck[i];
+        bi = ci[i];
+        bc = lane + 32 * i;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ok = __shfl_xor_sync(full, bk, off);
+      const int oi = __shfl_xor_sync(full, bi, off);
+      const int oc = __shfl_xor_sync(full, bc, off);
+      if (ok > bk || (ok == bk && oi < bi)) {
+        bk = ok;
+        bi = oi;
+        bc = oc;
+      }
+    }
+    if ((bc & 31) == lane) taken |= 1u << (bc >> 5);
+    float v = 0.f;
+#pragma unroll
+    for (int i = 0; i < kSmallTopkWarps; ++i)
+      if (i == (bc >> 5)) v = cs[i];
+    v = __shfl_sync(full, v, bc & 31);
+    if (lane == j) {
+      my_id = bi;
+      my_sc = v;
+    }
+  }
+  float total = lane < k ? my_sc : 0.f;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) total += __shfl_xor_sync(full, total, off);
+  if (lane < k) {
+    const float wgt = a.norm ? my_sc / total * a.scale : my_sc * a.scale;
+    a.ids[(size_t)t * k + lane] = my_id;
+    a.wts[(size_t)t * k + lane] = wgt;
+    if (a.ids_out) a.ids_out[(size_t)t * k + lane] = my_id;
+    if (a.wts_out) a.wts_out[(size_t)t * k + lane] = wgt;
+    atomicAdd(&a.counts[my_id], 1);
+    atomicOr(&a.bitmap[(size_t)my_id * a.W + (t >> 5)], 1u << (t & 31));
+  }
+}
+
 // Few tokens (T <= kRouterGemvMaxT): the 64 x 64 tiles of router_logits_kernel
 // would hold one or a few valid tokens and need a split-K sum, so instead one
 // CTA per expert reads its router row once (float4 loads, 256 threads
@@ -211,7 +396,10 @@ cudaError_t launch_router_topk(moe_handle* h, int T, int splits, const int32_t* 
                    h->cfg.routed_scaling_factor, h->cfg.norm_topk_prob, forced, h->ws.ids,
                    h->ws.wts, h->ws.counts, h->ws.bitmap, W, h->ws.status, ids_out, wts_out,
                    logits_out, h->cfg.n_group, h->cfg.topk_group};
-  router_topk_kernel<<<blocks, 256, 0, s>>>(a);
+  if (T <= kSmallTopkMaxT && forced == nullptr && h->cfg.n_group == 1)
+    router_topk_small_kernel<<<(T + 1) / 2, 256, 0, s>>>(a);
+  else
+    router_topk_kernel<<<blocks, 256, 0, s>>>(a);
   h->launches++;
   return cudaGetLastError();
 }
