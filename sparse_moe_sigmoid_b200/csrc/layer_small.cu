@@ -22,7 +22,7 @@
 // Measured against the phase kernels on one B200: the routing phases are
 // cheaper here, but the gate/up tiles stream 10-25% slower (decode T = 64:
 // 3.62 vs 3.38 ms; FP8 T = 16: 1.02 vs 0.87 ms; FP8 T = 1: 0.127 vs
-// 0.118 ms). It is therefore opt-in per handle (single_launch_max_tokens,
+// 0.112 ms). It is therefore opt-in per handle (single_launch_max_tokens,
 // default 0).
 //
 // Launch: cooperative (every CTA resident at once, or the launch fails), one

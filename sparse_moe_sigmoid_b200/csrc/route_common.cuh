@@ -302,17 +302,22 @@ __device__ __forceinline__ void quant_row_e4m3(const __nv_bfloat16* __restrict__
   }
 }
 
-// NC: read through the read-only path (the rows were written by an earlier
-// launch); the single-launch layer reads rows of its own launch coherently.
-template <bool NC = true>
-__device__ __forceinline__ void add_row8(float (&acc)[8], const uint16_t* p, float w) {
-  const uint4 v = NC ? __ldg(reinterpret_cast<const uint4*>(p)) : *reinterpret_cast<const uint4*>(p);
+// acc += w * (8 BF16 values packed in v)
+__device__ __forceinline__ void add_row8v(float (&acc)[8], const uint4 v, float w) {
   const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {  // BF16 -> fp32 is exact: the bits move up by 16
     acc[2 * i] = fmaf(w, __uint_as_float(u[i] << 16), acc[2 * i]);
     acc[2 * i + 1] = fmaf(w, __uint_as_float(u[i] & 0xFFFF0000u), acc[2 * i + 1]);
   }
+}
+
+// NC: read through the read-only path (the rows were written by an earlier
+// launch); the single-launch layer reads rows of its own launch coherently.
+template <bool NC = true>
+__device__ __forceinline__ void add_row8(float (&acc)[8], const uint16_t* p, float w) {
+  const uint4 v = NC ? __ldg(reinterpret_cast<const uint4*>(p)) : *reinterpret_cast<const uint4*>(p);
+  add_row8v(acc, v, w);
 }
 
 }  // namespace smoe
