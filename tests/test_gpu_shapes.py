@@ -49,6 +49,9 @@ CASES = [
     ("single_launch_no_norm", S(512, 256, 24, 4, 1, norm_topk_prob=False), 16, "bf16", 128),
     ("single_launch_grouped_fp8", S(512, 256, 24, 4, 1, n_group=4, topk_group=2), 16, "fp8",
      128),
+    # few tokens with fewer experts than the small-batch top-k's four warps
+    ("three_experts_few_tokens", S(512, 256, 3, 2, 1), 100, "bf16", 0),
+    ("one_expert_few_tokens", S(512, 256, 1, 1, 0), 50, "fp8", 0),
 ]
 
 
